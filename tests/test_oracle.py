@@ -1,0 +1,432 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: torch's
+float8_e4m3fn codec (an independent library implementation of E4M3FN),
+the OCP format table, hand-worked groups (tests/golden), closed forms,
+invariants of the definition and brute-force dequantize-then-matmul with
+numpy.  See oracle/fp8_oracle.c for the definition being pinned.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from blockwise_fp8_pretraining_b200 import synthetic as syn
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+G = 128
+
+
+# ------------------------------------------------------------------ helpers
+
+def torch_decode(codes):
+    """Library decode of E4M3FN codes (torch's float8_e4m3fn)."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def torch_encode(values):
+    """Library RNE cast to E4M3FN.  torch saturates to 448 only up to the
+    midpoint 464 and returns NaN beyond, so callers keep |v| <= 464."""
+    t = torch.from_numpy(np.ascontiguousarray(values, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def bits_of(values):
+    return np.asarray(values, dtype=np.float32).view(np.uint32)
+
+
+def to_bf16_bits(values):
+    t = torch.tensor(np.asarray(values, dtype=np.float32)).to(torch.bfloat16)
+    return syn.bf16_bits(t)
+
+
+def torch_quant_rowwise(x_bf16: torch.Tensor):
+    """The quantizer definition written with torch library primitives:
+    group amax, fp32 division by 448, fp32 division of each element, torch's
+    E4M3 cast.  Used only for data whose |x/s| stays within torch's
+    saturating range (always true for a group's own scale)."""
+    rows, cols = x_bf16.shape
+    xf = x_bf16.float().reshape(rows, cols // G, G)
+    amax = xf.abs().amax(dim=2)                              # [rows, groups]
+    s = amax / torch.tensor(448.0, dtype=torch.float32)
+    safe = torch.where(s == 0, torch.ones_like(s), s)
+    q = (xf / safe[:, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    q = torch.where((s == 0)[:, :, None], torch.zeros_like(q), q)
+    return q.reshape(rows, cols).numpy(), s.T.contiguous().numpy()
+
+
+def torch_quant_weight(w_bf16: torch.Tensor):
+    n, k = w_bf16.shape
+    wf = w_bf16.float().reshape(n // G, G, k // G, G)
+    amax = wf.abs().amax(dim=(1, 3))                         # [n/128, k/128]
+    s = amax / torch.tensor(448.0, dtype=torch.float32)
+    safe = torch.where(s == 0, torch.ones_like(s), s)
+    q = (wf / safe[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    q = torch.where((s == 0)[:, None, :, None], torch.zeros_like(q), q)
+    return q.reshape(n, k).numpy(), s.numpy()
+
+
+def dequant_rowwise(q, s):
+    """[rows, cols] values from codes and [cols/128, rows] scales."""
+    return torch_decode(q) * np.repeat(s.T.astype(np.float64), G, axis=1)
+
+
+def dequant_weight(q, s):
+    return torch_decode(q) * np.kron(s.astype(np.float64), np.ones((G, G)))
+
+
+def assert_close_to_bound(y, ref, bound, rel):
+    err = np.abs(y - ref)
+    assert np.all(err <= rel * bound + 1e-300), float((err / np.maximum(bound, 1e-300)).max())
+
+
+# -------------------------------------------------------------------- codec
+
+def test_decode_all_codes_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    ref = torch_decode(codes)
+    nan = np.isnan(ref)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))
+
+
+def test_decode_spot_values_from_format_table():
+    with open(os.path.join(GOLDEN, "e4m3_spot_values.txt")) as f:
+        rows = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    for code_s, val_s in rows:
+        got = oracle.e4m3_decode(np.array([int(code_s, 16)], np.uint8))[0]
+        want = float(val_s)
+        if np.isnan(want):
+            assert np.isnan(got), code_s
+        else:
+            assert got == want and np.signbit(got) == np.signbit(want), code_s
+
+
+def test_decode_grid_is_monotone_and_binade_spaced():
+    vals = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))   # 0x00..0x7E
+    assert np.all(np.diff(vals) > 0)
+    gaps = np.diff(vals)
+    # Subnormal steps and the step into the first normal binade are 2^-9;
+    # each later binade's step is twice the previous one.
+    assert np.all(gaps[:8] == 2.0 ** -9)
+    for e in range(1, 16):
+        seg = gaps[8 * e: 8 * e + 8]
+        assert seg.size > 0 and np.all(seg == 2.0 ** (e - 10)), e
+
+
+def test_encode_roundtrips_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_decode(codes).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(vals), codes)
+
+
+def test_encode_midpoints_tie_to_even_and_neighbours():
+    pos = np.arange(0x7F, dtype=np.uint8)
+    v = oracle.e4m3_decode(pos)
+    lo, hi = v[:-1], v[1:]
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (lo + hi) / 2)   # exact in fp32
+    even = np.where(pos[:-1] % 2 == 0, pos[:-1], pos[1:]).astype(np.uint8)
+    below = np.nextafter(mid, np.float32(0))
+    above = np.nextafter(mid, np.float32(np.inf))
+    for sign in (1.0, -1.0):
+        sb = np.uint8(0x80) if sign < 0 else np.uint8(0)
+        assert np.array_equal(oracle.e4m3_encode(sign * mid), even | sb)
+        assert np.array_equal(oracle.e4m3_encode(sign * below), pos[:-1] | sb)
+        assert np.array_equal(oracle.e4m3_encode(sign * above), pos[1:] | sb)
+        # the same decisions from the library cast
+        assert np.array_equal(torch_encode(sign * mid), even | sb)
+        assert np.array_equal(torch_encode(sign * below), pos[:-1] | sb)
+
+
+def test_encode_saturates_at_448():
+    big = np.array([448.0, 463.99, 464.0, 479.9, 480.0, 1e4, 1e30, 3.0e38], np.float32)
+    assert np.all(oracle.e4m3_encode(big) == 0x7E)
+    assert np.all(oracle.e4m3_encode(-big) == 0xFE)
+
+
+def test_encode_zero_and_tiny_keep_sign():
+    v = np.array([0.0, -0.0, 1e-30, -1e-30, 2.0 ** -10, -(2.0 ** -10), 1e-45, -1e-45], np.float32)
+    assert list(oracle.e4m3_encode(v)) == [0x00, 0x80, 0x00, 0x80, 0x00, 0x80, 0x00, 0x80]
+
+
+def test_encode_matches_torch_on_dense_sweep():
+    rng = np.random.default_rng(1)
+    mag = np.exp(rng.uniform(np.log(1e-6), np.log(464.0), 400_000)).astype(np.float32)
+    sign = np.where(rng.random(mag.size) < 0.5, -1, 1).astype(np.float32)
+    v = np.concatenate([mag * sign, rng.uniform(-464, 464, 100_000).astype(np.float32)])
+    assert np.array_equal(oracle.e4m3_encode(v), torch_encode(v))
+
+
+# --------------------------------------------------------------- quantizers
+
+def load_handworked():
+    scales, elems = [], []
+    with open(os.path.join(GOLDEN, "handworked_groups.txt")) as f:
+        for ln in f:
+            p = ln.split()
+            if not p or p[0].startswith("#"):
+                continue
+            if p[0] == "scale":
+                scales.append((int(p[1]), int(p[2]), int(p[3], 16)))
+            else:
+                elems.append((int(p[1]), int(p[2]), float(p[3]), int(p[4], 16)))
+    return scales, elems
+
+
+def test_handworked_groups_rowwise():
+    scales, elems = load_handworked()
+    x = np.zeros((2, 256), np.float32)
+    for r, c, v, _ in elems:
+        x[r, c] = v
+    xb = to_bf16_bits(x)
+    assert np.array_equal(oracle.bf16_to_float(xb), x)          # all exact in bf16
+    q, s = oracle.quantize_act_rowwise(xb)
+    want_q = np.zeros((2, 256), np.uint8)
+    for r, c, _, code in elems:
+        want_q[r, c] = code
+    assert np.array_equal(q, want_q)
+    assert s.shape == (2, 2)
+    for r, g, b in scales:
+        assert int(bits_of(s[g, r])) == b, (r, g)
+
+
+def test_handworked_groups_colwise_and_weight():
+    """The same groups placed along tokens (columns of X^T) and inside a
+    128x128 weight block must give the same codes and scales."""
+    scales, elems = load_handworked()
+    x = np.zeros((2, 256), np.float32)
+    for r, c, v, _ in elems:
+        x[r, c] = v
+    xt_bits = to_bf16_bits(x.T.copy())                           # [256, 2]
+    qT, s = oracle.quantize_act_colwise(xt_bits)                 # [2, 256], [2, 2]
+    q_row, s_row = oracle.quantize_act_rowwise(to_bf16_bits(x))
+    assert np.array_equal(qT, q_row)
+    assert np.array_equal(bits_of(s), bits_of(s_row))
+
+    # weight: row 0 group 0's 128 values spread over a 128x128 block, with
+    # an all-zero neighbour block.
+    w = np.zeros((128, 256), np.float32)
+    vals = x[0, :128]
+    w[np.arange(128), (np.arange(128) * 37) % 128] = vals
+    qw, sw = oracle.quantize_weight(to_bf16_bits(w))
+    assert sw.shape == (1, 2)
+    assert int(bits_of(sw[0, 0])) == 0x3F800000 and int(bits_of(sw[0, 1])) == 0
+    got = qw[np.arange(128), (np.arange(128) * 37) % 128]
+    assert np.array_equal(got, q_row[0, :128])
+    mask = np.ones_like(qw, bool)
+    mask[np.arange(128), (np.arange(128) * 37) % 128] = False
+    assert np.all(qw[mask] == 0)
+
+
+@pytest.mark.parametrize("maker", ["normal", "outlier", "student_t"])
+def test_rowwise_matches_torch_library_definition(maker):
+    if maker == "normal":
+        x = syn.normal_bf16((96, 1024), 1.0, syn.generator(3))
+    elif maker == "outlier":
+        x = syn.activation_bf16(130, 2048, 20, 30.0, syn.generator(4))
+    else:
+        x = syn.student_t_bf16((64, 2048), seed=5)
+    q, s = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    q_ref, s_ref = torch_quant_rowwise(x)
+    assert np.array_equal(bits_of(s), bits_of(s_ref))
+    assert np.array_equal(q, q_ref)
+
+
+def test_colwise_and_weight_match_torch_library_definition():
+    x = syn.activation_bf16(256, 384, 4, 50.0, syn.generator(6))
+    qT, s = oracle.quantize_act_colwise(syn.bf16_bits(x))
+    q_ref, s_ref = torch_quant_rowwise(x.T.contiguous())
+    assert np.array_equal(qT, q_ref)
+    assert np.array_equal(bits_of(s), bits_of(s_ref))
+
+    w = syn.normal_bf16((384, 256), 0.02, syn.generator(7))
+    qw, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    qw_ref, sw_ref = torch_quant_weight(w)
+    assert np.array_equal(qw, qw_ref)
+    assert np.array_equal(bits_of(sw), bits_of(sw_ref))
+
+
+def test_scaling_by_power_of_two_scales_s_and_keeps_codes():
+    x = syn.activation_bf16(32, 512, 4, 50.0, syn.generator(8))
+    q0, s0 = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    for k in (-20, -3, 1, 7):
+        xk = (x.float() * 2.0 ** k).to(torch.bfloat16)
+        assert torch.equal(xk.float(), x.float() * 2.0 ** k)     # exact
+        qk, sk = oracle.quantize_act_rowwise(syn.bf16_bits(xk))
+        assert np.array_equal(qk, q0)
+        assert np.array_equal(sk, s0 * np.float32(2.0 ** k))
+
+
+def test_row_permutation_permutes_outputs():
+    x = syn.activation_bf16(64, 256, 4, 50.0, syn.generator(9))
+    perm = torch.randperm(64, generator=syn.generator(10))
+    q, s = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    qp, sp = oracle.quantize_act_rowwise(syn.bf16_bits(x[perm]))
+    assert np.array_equal(qp, q[perm.numpy()])
+    assert np.array_equal(sp, s[:, perm.numpy()])
+
+
+def test_colwise_equals_rowwise_of_transpose():
+    x = syn.activation_bf16(384, 256, 4, 50.0, syn.generator(11))
+    qT, s = oracle.quantize_act_colwise(syn.bf16_bits(x))
+    qr, sr = oracle.quantize_act_rowwise(syn.bf16_bits(x.T.contiguous()))
+    assert np.array_equal(qT, qr) and np.array_equal(s, sr)
+
+
+def test_weight_of_transpose_is_transpose():
+    w = syn.normal_bf16((256, 384), 0.02, syn.generator(12))
+    q, s = oracle.quantize_weight(syn.bf16_bits(w))
+    qt, st = oracle.quantize_weight(syn.bf16_bits(w.T.contiguous()))
+    assert np.array_equal(qt, q.T) and np.array_equal(st, s.T)
+
+
+def test_all_zero_and_negative_zero_groups():
+    x = np.zeros((3, 256), np.float32)
+    x[1, :128] = -0.0
+    x[2, 128:] = 1.0
+    q, s = oracle.quantize_act_rowwise(to_bf16_bits(x))
+    assert np.all(q[:2] == 0) and np.all(q[2, :128] == 0)
+    assert np.all(s[:, :2] == 0) and s[0, 2] == 0
+    assert np.all(q[2, 128:] == 0x7E)
+
+
+def test_quantizer_bad_arguments():
+    with pytest.raises(ValueError):
+        oracle.quantize_act_rowwise(np.zeros((4, 100), np.uint16))
+    with pytest.raises(ValueError):
+        oracle.quantize_act_colwise(np.zeros((100, 128), np.uint16))
+    with pytest.raises(ValueError):
+        oracle.quantize_weight(np.zeros((128, 100), np.uint16))
+    inf = to_bf16_bits(np.full((1, 128), np.inf, np.float32))
+    with pytest.raises(ValueError):
+        oracle.quantize_act_rowwise(inf)
+
+
+def test_empty_rows():
+    q, s = oracle.quantize_act_rowwise(np.zeros((0, 256), np.uint16))
+    assert q.shape == (0, 256) and s.shape == (2, 0)
+
+
+# -------------------------------------------------------------------- GEMMs
+
+def _quant_case(seed, M, N, K):
+    g = syn.generator(seed)
+    x = syn.activation_bf16(M, K, 4, 30.0, g)
+    w = syn.normal_bf16((N, K), 0.02, g)
+    dy = syn.normal_bf16((M, N), 1e-3, g)
+    return x, w, dy
+
+
+def test_fprop_brute_force():
+    x, w, _ = _quant_case(20, 200, 384, 512)
+    xq, sx = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    wq, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    y, bound = oracle.gemm_fprop(xq, sx, wq, sw)
+    a = dequant_rowwise(xq, sx)
+    b = dequant_weight(wq, sw)
+    ref = a @ b.T
+    ref_bound = np.abs(a) @ np.abs(b).T
+    assert_close_to_bound(y, ref, ref_bound, 1e-12)
+    assert_close_to_bound(bound, ref_bound, ref_bound, 1e-12)
+    assert np.all(np.abs(y) <= bound * (1 + 1e-12))
+
+
+def test_dgrad_brute_force():
+    _, w, dy = _quant_case(21, 192, 384, 256)
+    dyq, sdy = oracle.quantize_act_rowwise(syn.bf16_bits(dy))
+    wq, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    dx, bound = oracle.gemm_dgrad(dyq, sdy, wq, sw)
+    a = dequant_rowwise(dyq, sdy)          # [M, N]
+    b = dequant_weight(wq, sw)             # [N, K]
+    ref = a @ b
+    ref_bound = np.abs(a) @ np.abs(b)
+    assert dx.shape == (192, 256)
+    assert_close_to_bound(dx, ref, ref_bound, 1e-12)
+    assert_close_to_bound(bound, ref_bound, ref_bound, 1e-12)
+
+
+def test_wgrad_brute_force():
+    x, _, dy = _quant_case(22, 384, 256, 384)
+    dyqT, sdyT = oracle.quantize_act_colwise(syn.bf16_bits(dy))   # [N, M]
+    xqT, sxT = oracle.quantize_act_colwise(syn.bf16_bits(x))      # [K, M]
+    dw, bound = oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT)
+    a = dequant_rowwise(dyqT, sdyT)        # [N, M]
+    b = dequant_rowwise(xqT, sxT)          # [K, M]
+    ref = a @ b.T
+    ref_bound = np.abs(a) @ np.abs(b).T
+    assert dw.shape == (256, 384)
+    assert_close_to_bound(dw, ref, ref_bound, 1e-12)
+    assert_close_to_bound(bound, ref_bound, ref_bound, 1e-12)
+
+
+def test_fprop_all_ones_closed_form():
+    ones = to_bf16_bits(np.ones((128, 128), np.float32))
+    xq, sx = oracle.quantize_act_rowwise(ones)
+    wq, sw = oracle.quantize_weight(ones)
+    assert np.all(xq == 0x7E) and np.all(wq == 0x7E)
+    s = Fraction(float(np.float32(1.0) / np.float32(448.0)))
+    want = 128 * (448 * s) ** 2
+    y, bound = oracle.gemm_fprop(xq, sx, wq, sw)
+    assert np.all(np.abs(y - float(want)) <= 2.0 ** -52 * float(want))
+    assert np.all(bound == y)
+
+
+def test_fprop_block_identity_weight():
+    x, _, _ = _quant_case(23, 128, 256, 256)
+    eye = to_bf16_bits(np.eye(256, dtype=np.float32))
+    xq, sx = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    wq, sw = oracle.quantize_weight(eye)
+    s_w = np.float32(1.0) / np.float32(448.0)
+    assert sw[0, 1] == 0 and sw[1, 0] == 0 and sw[0, 0] == s_w and sw[1, 1] == s_w
+    y, _ = oracle.gemm_fprop(xq, sx, wq, sw)
+    want = dequant_rowwise(xq, sx) * (448.0 * float(s_w))
+    assert np.all(np.abs(y - want) <= 1e-15 * np.abs(want))
+
+
+def test_fprop_single_nonzero_per_row():
+    rng = np.random.default_rng(24)
+    M, N, K = 128, 256, 384
+    xf = np.zeros((M, K), np.float32)
+    cols = rng.integers(0, K, M)
+    xf[np.arange(M), cols] = rng.normal(size=M).astype(np.float32)
+    w = syn.normal_bf16((N, K), 0.02, syn.generator(25))
+    xq, sx = oracle.quantize_act_rowwise(to_bf16_bits(xf))
+    wq, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    y, _ = oracle.gemm_fprop(xq, sx, wq, sw)
+    a = dequant_rowwise(xq, sx)
+    b = dequant_weight(wq, sw)
+    want = a[np.arange(M), cols][:, None] * b[:, cols].T
+    assert np.all(np.abs(y - want) <= 1e-15 * np.abs(want))
+
+
+def test_dgrad_equals_fprop_with_transposed_weight():
+    _, w, dy = _quant_case(26, 128, 256, 384)
+    dyq, sdy = oracle.quantize_act_rowwise(syn.bf16_bits(dy))
+    wq, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    wtq, swt = oracle.quantize_weight(syn.bf16_bits(w.T.contiguous()))
+    dx, b1 = oracle.gemm_dgrad(dyq, sdy, wq, sw)
+    y, b2 = oracle.gemm_fprop(dyq, sdy, wtq, swt)
+    assert np.array_equal(dx, y) and np.array_equal(b1, b2)
+
+
+def test_row_subset_matches_full():
+    x, w, dy = _quant_case(27, 256, 256, 256)
+    xq, sx = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    wq, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    y, b = oracle.gemm_fprop(xq, sx, wq, sw)
+    rows = [255, 0, 17, 17]
+    ys, bs = oracle.gemm_fprop(xq, sx, wq, sw, rows=rows)
+    assert np.array_equal(ys, y[rows]) and np.array_equal(bs, b[rows])
+    dyqT, sdyT = oracle.quantize_act_colwise(syn.bf16_bits(dy))
+    xqT, sxT = oracle.quantize_act_colwise(syn.bf16_bits(x))
+    dw, _ = oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT)
+    dws, _ = oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=[3, 200])
+    assert np.array_equal(dws, dw[[3, 200]])
