@@ -1,1 +1,29 @@
-"""Blockwise-E4M3 FP8 linear layer for B200 (sm_100a)."""
+"""Blockwise-E4M3 FP8 Transformer linear layer for NVIDIA B200 (sm_100a).
+
+The compute path is the CUDA library libfp8blk.so (C ABI in
+include/fp8blk.h); this package is its Python binding.  The functions carry
+the C entry points' names; see ``_abi`` for their arguments.  Nothing here falls back to a CPU or library implementation: calling
+a function without the built library raises.
+"""
+from ._abi import (  # noqa: F401
+    BOTH,
+    COLWISE,
+    MAX_CONTRACTION_FPROP,
+    ROWWISE,
+    Fp8Error,
+    fp8_block_gemm_dgrad,
+    fp8_block_gemm_fprop,
+    fp8_block_gemm_wgrad,
+    fp8_cast_e4m3_scaled,
+    fp8_clear_error,
+    fp8_get_error,
+    fp8_last_cuda_error,
+    fp8_quantize_act_1x128,
+    fp8_quantize_weight_128x128,
+    fp8_selftest_wait_timeout,
+    fp8_set_wait_timeout_ns,
+    fp8_status_string,
+    header_functions,
+    lib_path,
+    load,
+)

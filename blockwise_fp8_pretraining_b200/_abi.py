@@ -1,0 +1,254 @@
+"""ctypes binding of the C ABI in include/fp8blk.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls.  Tensors are
+torch CUDA tensors; outputs the caller does not pass are allocated with torch
+(device memory only: the library itself never allocates).  A non-zero status
+raises Fp8Error.  The library must have been built (``python -m
+blockwise_fp8_pretraining_b200.build``); there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+ROWWISE, COLWISE, BOTH = 1, 2, 3
+MAX_CONTRACTION_FPROP = 32768
+
+_lib = None
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        msg = f"{where}: {status_string(status)} (status {status})"
+        if status == 5:
+            msg += f": {fp8_last_cuda_error()}"
+        super().__init__(msg)
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/fp8blk.h declares."""
+    with open(_build.HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fp8_\w+)\s*\(", text, flags=re.M)
+
+
+def load() -> ctypes.CDLL:
+    """Load libfp8blk.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = lib_path()
+    if not os.path.exists(path):
+        raise OSError(f"{path} is missing: build it with python -m blockwise_fp8_pretraining_b200.build")
+    lib = ctypes.CDLL(path)
+    p, i64, i32, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int
+    sig = {
+        "fp8_quantize_act_1x128": [p, i64, i64, i32, p, p, p, p, p],
+        "fp8_quantize_weight_128x128": [p, i64, i64, p, p, p, p],
+        "fp8_block_gemm_fprop": [p, p, p, p, p, i64, i64, i64, p],
+        "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p],
+        "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p],
+        "fp8_get_error": [],
+        "fp8_clear_error": [],
+        "fp8_set_wait_timeout_ns": [ctypes.c_uint64],
+        "fp8_cast_e4m3_scaled": [p, ctypes.c_float, p, i64, p],
+        "fp8_selftest_wait_timeout": [p],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = st
+    lib.fp8_status_string.argtypes = [st]
+    lib.fp8_status_string.restype = ctypes.c_char_p
+    lib.fp8_last_cuda_error.argtypes = []
+    lib.fp8_last_cuda_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load().fp8_status_string(int(status)).decode()
+    except OSError:
+        return "library not loaded"
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise Fp8Error(status, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _want(t: torch.Tensor, dtype, shape, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _out(t, dtype, shape, device, name):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    return _want(t, dtype, shape, name)
+
+
+# ------------------------------------------------------------------ kernels
+
+def fp8_quantize_act_1x128(x, mode=BOTH, q_row=None, s_row=None, q_colT=None, s_col=None,
+                           stream=None):
+    """Quantize a bf16 activation [rows, cols].  Returns (q_row, s_row,
+    q_colT, s_col); entries of a grouping the mode leaves out are None."""
+    lib = load()
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    _want(x, torch.bfloat16, (rows, cols), "x")
+    dev = x.device
+    if mode & ROWWISE:
+        q_row = _out(q_row, torch.uint8, (rows, cols), dev, "q_row")
+        s_row = _out(s_row, torch.float32, (cols // 128, rows), dev, "s_row")
+    else:
+        q_row = s_row = None
+    if mode & COLWISE:
+        q_colT = _out(q_colT, torch.uint8, (cols, rows), dev, "q_colT")
+        s_col = _out(s_col, torch.float32, (rows // 128, cols), dev, "s_col")
+    else:
+        q_colT = s_col = None
+    _check(lib.fp8_quantize_act_1x128(_ptr(x), rows, cols, int(mode), _ptr(q_row), _ptr(s_row),
+                                      _ptr(q_colT), _ptr(s_col), _stream(stream)),
+           "fp8_quantize_act_1x128")
+    return q_row, s_row, q_colT, s_col
+
+
+def fp8_quantize_weight_128x128(w, wq=None, sw=None, wqT=None, transposed=True, stream=None):
+    """Quantize a bf16 weight [n, k] in 128x128 blocks.  Returns (wq, sw, wqT);
+    wqT is None when transposed is False and no buffer is passed."""
+    lib = load()
+    if w.dtype != torch.bfloat16 or w.dim() != 2:
+        raise TypeError("w must be a 2-D bfloat16 tensor")
+    n, k = w.shape
+    _want(w, torch.bfloat16, (n, k), "w")
+    wq = _out(wq, torch.uint8, (n, k), w.device, "wq")
+    sw = _out(sw, torch.float32, (n // 128, k // 128), w.device, "sw")
+    if wqT is not None or transposed:
+        wqT = _out(wqT, torch.uint8, (k, n), w.device, "wqT")
+    _check(lib.fp8_quantize_weight_128x128(_ptr(w), n, k, _ptr(wq), _ptr(sw), _ptr(wqT),
+                                           _stream(stream)),
+           "fp8_quantize_weight_128x128")
+    return wq, sw, wqT
+
+
+def fp8_block_gemm_fprop(xq, sx, wq, sw, y=None, stream=None):
+    """Y[M, N] = X W^T (bf16) from X codes [M, K] / scales [K/128, M] and W
+    codes [N, K] / scales [N/128, K/128]."""
+    lib = load()
+    M, K = xq.shape
+    N = wq.shape[0]
+    _want(xq, torch.uint8, (M, K), "xq")
+    _want(sx, torch.float32, (K // 128, M), "sx")
+    _want(wq, torch.uint8, (N, K), "wq")
+    _want(sw, torch.float32, (N // 128, K // 128), "sw")
+    y = _out(y, torch.bfloat16, (M, N), xq.device, "y")
+    _check(lib.fp8_block_gemm_fprop(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K,
+                                    _stream(stream)),
+           "fp8_block_gemm_fprop")
+    return y
+
+
+def fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=None, stream=None):
+    """dX[M, K] = dY W (bf16) from dY codes [M, N] / scales [N/128, M], the
+    transposed weight codes [K, N] and the weight scales [N/128, K/128]."""
+    lib = load()
+    M, N = dyq.shape
+    K = wqT.shape[0]
+    _want(dyq, torch.uint8, (M, N), "dyq")
+    _want(sdy, torch.float32, (N // 128, M), "sdy")
+    _want(wqT, torch.uint8, (K, N), "wqT")
+    _want(sw, torch.float32, (N // 128, K // 128), "sw")
+    dx = _out(dx, torch.bfloat16, (M, K), dyq.device, "dx")
+    _check(lib.fp8_block_gemm_dgrad(_ptr(dyq), _ptr(sdy), _ptr(wqT), _ptr(sw), _ptr(dx), M, N, K,
+                                    _stream(stream)),
+           "fp8_block_gemm_dgrad")
+    return dx
+
+
+def fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=None, stream=None):
+    """dW[N, K] = dY^T X (bf16) from along-token codes: dY^T [N, M] / scales
+    [M/128, N] and X^T [K, M] / scales [M/128, K]."""
+    lib = load()
+    N, M = dyqT.shape
+    K = xqT.shape[0]
+    _want(dyqT, torch.uint8, (N, M), "dyqT")
+    _want(sdyT, torch.float32, (M // 128, N), "sdyT")
+    _want(xqT, torch.uint8, (K, M), "xqT")
+    _want(sxT, torch.float32, (M // 128, K), "sxT")
+    dw = _out(dw, torch.bfloat16, (N, K), dyqT.device, "dw")
+    _check(lib.fp8_block_gemm_wgrad(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw), N, K, M,
+                                    _stream(stream)),
+           "fp8_block_gemm_wgrad")
+    return dw
+
+
+def fp8_get_error() -> int:
+    return int(load().fp8_get_error())
+
+
+def fp8_clear_error() -> None:
+    _check(load().fp8_clear_error(), "fp8_clear_error")
+
+
+def fp8_set_wait_timeout_ns(ns: int) -> None:
+    _check(load().fp8_set_wait_timeout_ns(int(ns)), "fp8_set_wait_timeout_ns")
+
+
+def fp8_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def fp8_last_cuda_error() -> str:
+    try:
+        return load().fp8_last_cuda_error().decode()
+    except OSError:
+        return ""
+
+
+
+def fp8_cast_e4m3_scaled(x, scale: float, q=None, stream=None):
+    lib = load()
+    n = x.numel()
+    _want(x, torch.float32, tuple(x.shape), "x")
+    q = _out(q, torch.uint8, tuple(x.shape), x.device, "q")
+    _check(lib.fp8_cast_e4m3_scaled(_ptr(x), ctypes.c_float(scale), _ptr(q), n, _stream(stream)),
+           "fp8_cast_e4m3_scaled")
+    return q
+
+
+def fp8_selftest_wait_timeout(stream=None) -> None:
+    _check(load().fp8_selftest_wait_timeout(_stream(stream)), "fp8_selftest_wait_timeout")

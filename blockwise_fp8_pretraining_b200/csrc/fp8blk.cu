@@ -1,0 +1,320 @@
+// C ABI of the blockwise-E4M3 FP8 linear-layer library (see include/fp8blk.h
+// for the contract of every entry point).  Host code here only checks
+// arguments, builds TMA tensor maps and launches kernels on the caller's
+// stream; it never allocates or synchronizes (except fp8_get_error /
+// fp8_clear_error, which read or reset the device error word).
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/fp8blk.h"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+static_assert(fp8blk::kErrTimeout == static_cast<unsigned int>(FP8_ERR_TIMEOUT),
+              "device time-out code must match the C ABI");
+
+namespace {
+
+using namespace fp8blk;
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_gemm_attr_done[kMaxDevices];
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Text of the last CUDA failure this thread saw (for fp8_last_cuda_error).
+thread_local char g_detail[256] = "";
+
+fp8_status cuda_fail(const char* where, cudaError_t e) {
+    snprintf(g_detail, sizeof g_detail, "%s: %s (%d)", where, cudaGetErrorString(e), static_cast<int>(e));
+    return FP8_ERR_CUDA;
+}
+
+inline fp8_status last_launch_status(const char* where) {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FP8_OK : cuda_fail(where, e);
+}
+
+fp8_status current_device(int* dev) {
+    const cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (*dev < 0 || *dev >= kMaxDevices) return cuda_fail("device ordinal out of range", cudaErrorInvalidDevice);
+    return FP8_OK;
+}
+
+fp8_status sm_count(int dev, int* out) {
+    int n = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        const cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
+        g_sm_count[dev].store(n, std::memory_order_relaxed);
+    }
+    *out = n;
+    return FP8_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::atomic<void*> fn{nullptr};
+    void* f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        cudaDriverEntryPointQueryResult q;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) {
+            snprintf(g_detail, sizeof g_detail, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled): %s, query %d",
+                     cudaGetErrorString(e), static_cast<int>(q));
+            return nullptr;
+        }
+        fn.store(f, std::memory_order_release);
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+}
+
+// Row-major [rows, cols] byte matrix, boxes of box_rows x 128 bytes in the
+// 128-byte swizzle the MMA descriptors expect; out-of-range rows read as 0.
+fp8_status make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t cols,
+                            int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return FP8_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estride[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides,
+                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled: CUresult %d", static_cast<int>(r));
+        return FP8_ERR_CUDA;
+    }
+    return FP8_OK;
+}
+
+// Shared launcher of the three GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
+// codes, both K-major; scales described by `p`.
+template <int SCALE>
+fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, gemm::Params p, cudaStream_t stream) {
+    int dev = 0, sms = 0;
+    fp8_status st = current_device(&dev);
+    if (st != FP8_OK) return st;
+    if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
+
+    const int flag = 1 << SCALE;
+    if ((g_gemm_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
+        const cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   gemm::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
+        g_gemm_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
+    }
+
+    CUtensorMap ma, mb;
+    if ((st = make_operand_map(&ma, a, p.M, p.K, gemm::BM)) != FP8_OK) return st;
+    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN)) != FP8_OK) return st;
+
+    p.tiles_m = static_cast<int>((p.M + gemm::BM - 1) / gemm::BM);
+    p.tiles_n = static_cast<int>((p.N + gemm::BN - 1) / gemm::BN);
+    p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    gemm::gemm_kernel<SCALE><<<grid, gemm::THREADS, gemm::SMEM_BYTES, stream>>>(ma, mb, p);
+    return last_launch_status("gemm launch");
+}
+
+bool dims_ok_gemm(int64_t M, int64_t N, int64_t K, bool m_positive) {
+    if (M < 0 || N <= 0 || K <= 0) return false;
+    if (m_positive && M == 0) return false;
+    if (M % 128 || N % 128 || K % 128) return false;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return false;
+    if (static_cast<int64_t>((M + 127) / 128) * ((N + 255) / 256) > kMaxDim) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8_status fp8_quantize_act_1x128(const void* x_bf16, int64_t rows, int64_t cols, int mode,
+                                  uint8_t* q_row, float* s_row, uint8_t* q_colT, float* s_col,
+                                  void* stream) {
+    if (mode != FP8_ROWWISE && mode != FP8_COLWISE && mode != FP8_BOTH) return FP8_ERR_MODE;
+    if (rows < 0 || cols < 0 || cols % 128 != 0 || rows > kMaxDim || cols > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if ((mode & FP8_COLWISE) && rows % 128 != 0) return FP8_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    if (!x_bf16) return FP8_ERR_NULL;
+    if ((mode & FP8_ROWWISE) && (!q_row || !s_row)) return FP8_ERR_NULL;
+    if ((mode & FP8_COLWISE) && (!q_colT || !s_col)) return FP8_ERR_NULL;
+    if (!aligned16(x_bf16)) return FP8_ERR_ALIGN;
+    if ((mode & FP8_ROWWISE) && (!aligned16(q_row) || !aligned16(s_row))) return FP8_ERR_ALIGN;
+    if ((mode & FP8_COLWISE) && (!aligned16(q_colT) || !aligned16(s_col))) return FP8_ERR_ALIGN;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint4* x = static_cast<const uint4*>(x_bf16);
+    if (mode == FP8_ROWWISE) {
+        int dev = 0, sms = 0;
+        fp8_status st = current_device(&dev);
+        if (st != FP8_OK) return st;
+        if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
+        constexpr int kUnroll = 4;
+        const int64_t groups = cols / 128;
+        const int64_t units = rows * groups;
+        const int64_t warps_needed = (units + 2 * kUnroll - 1) / (2 * kUnroll);
+        int64_t blocks = (warps_needed + 7) / 8;
+        const int64_t cap = static_cast<int64_t>(sms) * 8;
+        if (blocks > cap) blocks = cap;
+        quant_rowwise_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            x, units, rows, groups, reinterpret_cast<uint2*>(q_row), s_row);
+        return last_launch_status("row-wise quantize launch");
+    }
+    const int64_t tiles = (rows / 128) * (cols / 128);
+    if (tiles > kMaxDim) return FP8_ERR_SHAPE;
+    if (mode == FP8_COLWISE)
+        quant_tile_kernel<kTileColwise><<<static_cast<unsigned>(tiles), 256, 0, s>>>(
+            x, rows, cols, nullptr, nullptr, q_colT, s_col);
+    else
+        quant_tile_kernel<kTileBoth><<<static_cast<unsigned>(tiles), 256, 0, s>>>(
+            x, rows, cols, q_row, s_row, q_colT, s_col);
+    return last_launch_status("tile quantize launch");
+}
+
+fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k, uint8_t* wq,
+                                       float* sw, uint8_t* wqT, void* stream) {
+    if (n < 0 || k < 0 || n % 128 || k % 128 || n > kMaxDim || k > kMaxDim) return FP8_ERR_SHAPE;
+    if (n == 0 || k == 0) return FP8_OK;
+    if (!w_bf16 || !wq || !sw) return FP8_ERR_NULL;
+    if (!aligned16(w_bf16) || !aligned16(wq) || !aligned16(sw) || (wqT && !aligned16(wqT)))
+        return FP8_ERR_ALIGN;
+    const int64_t tiles = (n / 128) * (k / 128);
+    if (tiles > kMaxDim) return FP8_ERR_SHAPE;
+    quant_tile_kernel<kTileWeight><<<static_cast<unsigned>(tiles), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(w_bf16), n, k, wq, nullptr, wqT, sw);
+    return last_launch_status("weight quantize launch");
+}
+
+fp8_status fp8_block_gemm_fprop(const uint8_t* xq, const float* sx, const uint8_t* wq,
+                                const float* sw, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+    if (!dims_ok_gemm(M, N, K, false) || K > FP8_MAX_CONTRACTION_FPROP) return FP8_ERR_SHAPE;
+    if (M == 0) return FP8_OK;
+    if (!xq || !sx || !wq || !sw || !y_bf16) return FP8_ERR_NULL;
+    if (!aligned16(xq) || !aligned16(sx) || !aligned16(wq) || !aligned16(sw) || !aligned16(y_bf16))
+        return FP8_ERR_ALIGN;
+    gemm::Params p{};
+    p.sa = sx;
+    p.sa_ld = M;                 // sx [K/128, M]
+    p.sb = sw;
+    p.sb_sn = K / 128;           // sw [N/128, K/128]
+    p.sb_sk = 1;
+    p.out = static_cast<__nv_bfloat16*>(y_bf16);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    return launch_gemm<gemm::kScaleRowBlock>(xq, wq, p, static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_block_gemm_dgrad(const uint8_t* dyq, const float* sdy, const uint8_t* wqT,
+                                const float* sw, void* dx_bf16, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+    if (!dims_ok_gemm(M, K, N, false) || N > FP8_MAX_CONTRACTION_FPROP) return FP8_ERR_SHAPE;
+    if (M == 0) return FP8_OK;
+    if (!dyq || !sdy || !wqT || !sw || !dx_bf16) return FP8_ERR_NULL;
+    if (!aligned16(dyq) || !aligned16(sdy) || !aligned16(wqT) || !aligned16(sw) || !aligned16(dx_bf16))
+        return FP8_ERR_ALIGN;
+    gemm::Params p{};
+    p.sa = sdy;
+    p.sa_ld = M;                 // sdy [N/128, M]
+    p.sb = sw;                   // s_b(output block kb, slab nb) = sw[nb][kb]
+    p.sb_sn = 1;
+    p.sb_sk = K / 128;
+    p.out = static_cast<__nv_bfloat16*>(dx_bf16);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(K);
+    p.K = static_cast<int>(N);
+    return launch_gemm<gemm::kScaleRowBlock>(dyq, wqT, p, static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_block_gemm_wgrad(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
+                                const float* sxT, void* dw_bf16, int64_t N, int64_t K, int64_t M,
+                                void* stream) {
+    if (!dims_ok_gemm(N, K, M, true)) return FP8_ERR_SHAPE;
+    if (!dyqT || !sdyT || !xqT || !sxT || !dw_bf16) return FP8_ERR_NULL;
+    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_bf16))
+        return FP8_ERR_ALIGN;
+    gemm::Params p{};
+    p.sa = sdyT;
+    p.sa_ld = N;                 // sdyT [M/128, N]
+    p.sb = sxT;
+    p.sb_ld = K;                 // sxT [M/128, K]
+    p.out = static_cast<__nv_bfloat16*>(dw_bf16);
+    p.M = static_cast<int>(N);
+    p.N = static_cast<int>(K);
+    p.K = static_cast<int>(M);
+    return launch_gemm<gemm::kScaleOuter>(dyqT, xqT, p, static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_get_error(void) {
+    unsigned int v = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail("cudaDeviceSynchronize", e);
+    e = cudaMemcpyFromSymbol(&v, fp8blk::g_error_word, sizeof v);
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyFromSymbol", e);
+    return static_cast<fp8_status>(v);
+}
+
+fp8_status fp8_clear_error(void) {
+    const unsigned int zero = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail("cudaDeviceSynchronize", e);
+    e = cudaMemcpyToSymbol(fp8blk::g_error_word, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyToSymbol", e);
+    return FP8_OK;
+}
+
+const char* fp8_last_cuda_error(void) { return g_detail; }
+
+fp8_status fp8_set_wait_timeout_ns(uint64_t ns) {
+    g_wait_ns.store(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);
+    return FP8_OK;
+}
+
+const char* fp8_status_string(fp8_status status) {
+    switch (status) {
+        case FP8_OK: return "ok";
+        case FP8_ERR_NULL: return "a required pointer is NULL";
+        case FP8_ERR_SHAPE: return "unsupported shape";
+        case FP8_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case FP8_ERR_MODE: return "unknown mode";
+        case FP8_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case FP8_ERR_TIMEOUT: return "a bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+fp8_status fp8_cast_e4m3_scaled(const float* x, float scale, uint8_t* q, int64_t n, void* stream) {
+    if (n < 0) return FP8_ERR_SHAPE;
+    if (n == 0) return FP8_OK;
+    if (!x || !q) return FP8_ERR_NULL;
+    const int64_t blocks = (n + 255) / 256;
+    if (blocks > kMaxDim) return FP8_ERR_SHAPE;
+    cast_e4m3_scaled_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        x, scale, q, n);
+    return last_launch_status("cast launch");
+}
+
+fp8_status fp8_selftest_wait_timeout(void* stream) {
+    wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        g_wait_ns.load(std::memory_order_relaxed), static_cast<unsigned int>(FP8_ERR_TIMEOUT));
+    return last_launch_status("wait self-test launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,381 @@
+// FP8 block-scaled GEMM on tcgen05 tensor cores (sm_100a).
+//
+//   C[i, j] = sum_t  s_a(t, i) * s_b(t, j) * P_t[i, j],
+//   P_t[i, j] = sum_{k in slab t} A[i, k] * B[j, k]      (E4M3 codes)
+//
+// with 128-wide contraction slabs t and BF16 output.  This is the promotion
+// scheme of the DeepSeek-V3 FP8 recipe that the Puro-2B tech report's
+// related-work section (part 7/7, section 5) cites: every slab's partial sum
+// leaves the tensor core in FP32 and is scaled before it joins the running
+// FP32 accumulator.
+//
+// Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
+//   warp 0      TMA producer: A tile 128 x 128 B and B tile 256 x 128 B per
+//               slab into a 4-deep ring of 128-byte-swizzled stages, plus the
+//               slab's scale vectors into an 8-deep ring (plain bulk copies;
+//               no multicast anywhere).
+//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=32, E4M3 ->
+//               F32) per slab into one of two 256-column TMEM buffers, fresh
+//               for every slab; commits free the smem stage and publish the
+//               TMEM buffer.
+//   warps 2, 3  idle (they complete warpgroup 0, which gives registers away)
+//   warps 4..11 promotion + epilogue: each thread owns one output row (TMEM
+//               lane) and 128 columns, pulls the slab partials with
+//               tcgen05.ld, does acc = fma(s_a * s_b, P, acc) in registers,
+//               releases the TMEM buffer, and after the last slab rounds to
+//               BF16 and stores.  TMEM double buffering lets promotion of
+//               slab t overlap the MMAs of slab t+1.
+// Scale modes:
+//   kScaleRowBlock (fprop, dgrad): s_a is per output row (1x128 activation
+//     groups), s_b per 128-column block of the weight (128x128 blocks), so
+//     the coefficient is one number per thread per slab.
+//   kScaleOuter (wgrad): both operands are grouped along tokens, so the
+//     coefficient is the outer product s_a(t, i) * s_b(t, j).
+// Every mbarrier wait is bounded in time (see mbar_wait); on a time-out the
+// block stops issuing work, drains the copies and MMAs it has in flight,
+// frees its tensor memory and exits.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace fp8blk {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;              // one quantization slab
+constexpr int UMMA_K = 32;           // K of one kind::f8f6f4 MMA
+constexpr int STAGES = 4;
+constexpr int SSTAGES = 8;
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARP0 = 4;         // first epilogue warp (warpgroups 1 and 2)
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
+// Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup
+// 0 drops to 40 and the two epilogue warpgroups rise to 232:
+// 128 x 40 + 256 x 232 = 64512.
+constexpr int REGS_LAUNCH = 168;
+constexpr int REGS_PRODUCER = 40;
+constexpr int REGS_EPILOGUE = 232;
+static_assert(128 * REGS_PRODUCER + 256 * REGS_EPILOGUE <= THREADS * REGS_LAUNCH,
+              "register split exceeds the launch allocation");
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int SCALE_SLOT_BYTES = (BM + BN) * 4;
+constexpr int MAX_KB = 256;          // slabs of a fprop/dgrad contraction
+constexpr int SB_REGS = MAX_KB / 32;
+
+constexpr int OFF_SCALES = STAGES * STAGE_BYTES;
+constexpr int OFF_BARS = OFF_SCALES + SSTAGES * SCALE_SLOT_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 * SSTAGES + 1;
+constexpr int OFF_TMEM_SLOT = OFF_BARS + NUM_BARS * 8;
+constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
+
+constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
+
+enum ScaleMode : int { kScaleRowBlock = 0, kScaleOuter = 1 };
+
+struct Params {
+    const float* sa;        // s_a(t, i) = sa[t * sa_ld + i]
+    int64_t sa_ld;
+    const float* sb;        // row-block: s_b(nb, t) = sb[nb * sb_sn + t * sb_sk]
+    int64_t sb_sn, sb_sk;   // outer:     s_b(t, j)  = sb[t * sb_ld + j]
+    int64_t sb_ld;
+    __nv_bfloat16* out;     // [M, N]
+    int M, N, K;            // output rows, output columns, contraction
+    int tiles_m, tiles_n;
+    uint64_t wait_ns;
+};
+
+struct Bars {
+    uint32_t full, empty, tfull, tempty, sfull, sempty, drain;
+    __device__ __forceinline__ uint32_t full_(int s) const { return full + 8 * s; }
+    __device__ __forceinline__ uint32_t empty_(int s) const { return empty + 8 * s; }
+    __device__ __forceinline__ uint32_t tfull_(int b) const { return tfull + 8 * b; }
+    __device__ __forceinline__ uint32_t tempty_(int b) const { return tempty + 8 * b; }
+    __device__ __forceinline__ uint32_t sfull_(int s) const { return sfull + 8 * s; }
+    __device__ __forceinline__ uint32_t sempty_(int s) const { return sempty + 8 * s; }
+};
+
+// Wait without the abort check, used only while draining after a time-out.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return;
+    }
+}
+
+// s_b of slab kb from the 8 per-lane registers (lane j holds slab j + 32 r).
+__device__ __forceinline__ float pick_sb(const float (&regs)[SB_REGS], int kb) {
+    float v = 0.0f;
+#pragma unroll
+    for (int r = 0; r < SB_REGS; ++r)
+        if ((kb >> 5) == r) v = regs[r];
+    return __shfl_sync(0xffffffffu, v, kb & 31);
+}
+
+__device__ __forceinline__ void load_sb(float (&regs)[SB_REGS], const Params& p, int tile,
+                                        int half, int num_kb, int lane) {
+    const int total = p.tiles_m * p.tiles_n;
+    const int nb_count = p.N / 128;
+    int nb = -1;
+    if (tile < total) nb = (tile % p.tiles_n) * (BN / 128) + half;
+#pragma unroll
+    for (int r = 0; r < SB_REGS; ++r) {
+        const int kb = lane + 32 * r;
+        regs[r] = (nb >= 0 && nb < nb_count && kb < num_kb) ? __ldg(p.sb + nb * p.sb_sn + kb * p.sb_sk)
+                                                           : 0.0f;
+    }
+}
+
+template <int SCALE>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_kb = p.K / BK;
+    const int total_tiles = p.tiles_m * p.tiles_n;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+
+    Bars bars;
+    bars.full = sbase + OFF_BARS;
+    bars.empty = bars.full + 8 * STAGES;
+    bars.tfull = bars.empty + 8 * STAGES;
+    bars.tempty = bars.tfull + 16;
+    bars.sfull = bars.tempty + 16;
+    bars.sempty = bars.sfull + 8 * SSTAGES;
+    bars.drain = bars.sempty + 8 * SSTAGES;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bars.full_(s), 1);
+            mbar_init(bars.empty_(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bars.tfull_(b), 1);
+            mbar_init(bars.tempty_(b), EPI_WARPS);
+        }
+        for (int s = 0; s < SSTAGES; ++s) {
+            mbar_init(bars.sfull_(s), 1);
+            mbar_init(bars.sempty_(s), EPI_WARPS);
+        }
+        mbar_init(bars.drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(sbase + OFF_TMEM_SLOT, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
+
+    if (warp < EPI_WARP0) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
+      if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int it = 0;    // slabs whose operand tiles were requested
+            int its = 0;   // slabs whose scale vectors were requested
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                const int m0 = (tile / p.tiles_n) * BM;
+                const int n0 = (tile % p.tiles_n) * BN;
+                const uint32_t sb_bytes =
+                    (SCALE == kScaleOuter) ? static_cast<uint32_t>(min(BN, p.N - n0)) * 4u : 0u;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(bars.empty_(s), ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = sbase + s * STAGE_BYTES;
+                    mbar_arrive_expect_tx(bars.full_(s), STAGE_BYTES);
+                    tma_load_2d(a_dst, &tmA, kb * BK, m0, bars.full_(s));
+                    tma_load_2d(a_dst + A_BYTES, &tmB, kb * BK, n0, bars.full_(s));
+                    ++it;
+
+                    const int ss = its % SSTAGES;
+                    if (!mbar_wait(bars.sempty_(ss), ((its / SSTAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t slot = sbase + OFF_SCALES + ss * SCALE_SLOT_BYTES;
+                    mbar_arrive_expect_tx(bars.sfull_(ss), BM * 4 + sb_bytes);
+                    bulk_load(slot, p.sa + static_cast<int64_t>(kb) * p.sa_ld + m0, BM * 4,
+                              bars.sfull_(ss));
+                    if (SCALE == kScaleOuter)
+                        bulk_load(slot + BM * 4, p.sb + static_cast<int64_t>(kb) * p.sb_ld + n0,
+                                  sb_bytes, bars.sfull_(ss));
+                    ++its;
+                }
+            }
+            if (!ok) {
+                // Let every copy already requested land before the block exits.
+                for (int j = max(0, it - STAGES); j < it; ++j)
+                    drain_wait(bars.full_(j % STAGES), (j / STAGES) & 1, p.wait_ns);
+                for (int j = max(0, its - SSTAGES); j < its; ++j)
+                    drain_wait(bars.sfull_(j % SSTAGES), (j / SSTAGES) & 1, p.wait_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int buf = it & 1;
+                    if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    const int s = it % STAGES;
+                    if (!mbar_wait(bars.full_(s), (it / STAGES) & 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = sbase + s * STAGE_BYTES;
+                    const uint64_t a_desc = smem_desc_k128_sw128(a_addr);
+                    const uint64_t b_desc = smem_desc_k128_sw128(a_addr + A_BYTES);
+                    const uint32_t d_tmem = tmem_base + buf * BN;
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        // +32 bytes along K inside the swizzled 128-byte row
+                        const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
+                        mma_f8(d_tmem, a_desc + adv, b_desc + adv, IDESC, k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bars.empty_(s));
+                    mma_commit(bars.tfull_(buf));
+                }
+            }
+            // All MMAs of this thread done before the block may free TMEM.
+            mma_commit(bars.drain);
+            drain_wait(bars.drain, 0, p.wait_ns);
+        }
+        __syncwarp();
+      }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_EPILOGUE));
+        // ----------------------------------------------- promotion + epilogue
+        const int ew = warp - EPI_WARP0;
+        const int quarter = warp & 3;          // TMEM lanes this warp may read
+        const int half = ew >> 2;              // which 128 of the 256 columns
+        const int row_in_tile = quarter * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+
+        float sb_cur[SB_REGS], sb_next[SB_REGS];
+        if (SCALE == kScaleRowBlock) load_sb(sb_cur, p, blockIdx.x, half, num_kb, lane);
+
+        float acc[128];
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+            const int m0 = (tile / p.tiles_n) * BM;
+            const int n0 = (tile % p.tiles_n) * BN;
+            if (SCALE == kScaleRowBlock) load_sb(sb_next, p, tile + gridDim.x, half, num_kb, lane);
+#pragma unroll
+            for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int buf = it & 1;
+                const int ss = it % SSTAGES;
+                bool got = mbar_wait(bars.tfull_(buf), (it >> 1) & 1, abort_flag, p.wait_ns, kErrTimeout);
+                got = got && mbar_wait(bars.sfull_(ss), (it / SSTAGES) & 1, abort_flag, p.wait_ns, kErrTimeout);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float* slot =
+                    reinterpret_cast<const float*>(smem + OFF_SCALES + ss * SCALE_SLOT_BYTES);
+                const float sa = slot[row_in_tile];
+                const uint32_t taddr = lane_base + buf * BN + half * 128;
+                if (SCALE == kScaleRowBlock) {
+                    const float c = sa * pick_sb(sb_cur, kb);
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(taddr + ch * 32, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            acc[ch * 32 + j] = fmaf(c, __uint_as_float(r[j]), acc[ch * 32 + j]);
+                    }
+                } else {
+                    const float* sbv = slot + BM + half * 128;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(taddr + ch * 32, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 b4 = *reinterpret_cast<const float4*>(sbv + ch * 32 + j);
+                            acc[ch * 32 + j + 0] = fmaf(sa * b4.x, __uint_as_float(r[j + 0]), acc[ch * 32 + j + 0]);
+                            acc[ch * 32 + j + 1] = fmaf(sa * b4.y, __uint_as_float(r[j + 1]), acc[ch * 32 + j + 1]);
+                            acc[ch * 32 + j + 2] = fmaf(sa * b4.z, __uint_as_float(r[j + 2]), acc[ch * 32 + j + 2]);
+                            acc[ch * 32 + j + 3] = fmaf(sa * b4.w, __uint_as_float(r[j + 3]), acc[ch * 32 + j + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bars.tempty_(buf));
+                    mbar_arrive(bars.sempty_(ss));
+                }
+            }
+            if (!ok) break;
+
+            // BF16 round-to-nearest-even and store of this thread's row.
+            const int col0 = n0 + half * 128;
+            if (col0 < p.N) {
+                __nv_bfloat16* dst = p.out + static_cast<int64_t>(m0 + row_in_tile) * p.N + col0;
+#pragma unroll
+                for (int j = 0; j < 128; j += 8) {
+                    uint4 o;
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+                    __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+                    o.x = *reinterpret_cast<uint32_t*>(&h0);
+                    o.y = *reinterpret_cast<uint32_t*>(&h1);
+                    o.z = *reinterpret_cast<uint32_t*>(&h2);
+                    o.w = *reinterpret_cast<uint32_t*>(&h3);
+                    *reinterpret_cast<uint4*>(dst + j) = o;
+                }
+            }
+            if (SCALE == kScaleRowBlock) {
+#pragma unroll
+                for (int r = 0; r < SB_REGS; ++r) sb_cur[r] = sb_next[r];
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace gemm
+}  // namespace fp8blk

@@ -1,0 +1,201 @@
+/*
+ * fp8blk.h - C ABI of the blockwise-E4M3 FP8 linear-layer library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * The Puro-2B-Base model card (friendli.ai; repeated on the alphaneural.io
+ * card), in the training-setup paragraph under the Phase 1 / Phase 2 setting
+ * table, says the main Transformer linear-layer GEMMs run in blockwise E4M3
+ * FP8 and that numerically sensitive operations, master weights and
+ * optimizer state stay in BF16/FP32.  The tech report (part 7/7, section 5,
+ * related work) ties this to the FP8 mixed-precision recipe of DeepSeek-V3.
+ * The pages fix no block size or scale format; this library defines them:
+ *
+ *   - activations: groups of 1x128 consecutive elements along the GEMM's
+ *     contraction dimension; weights: 128x128 blocks;
+ *   - scale s = amax / 448 as an IEEE float32 division, stored as float32
+ *     (the dequantization multiplier; an all-zero group stores 0);
+ *   - code = E4M3FN(x / s): IEEE float32 division, then round-to-nearest-
+ *     even onto the OCP E4M3FN grid, saturating at +-448, sign kept
+ *     (a negative value that rounds to zero is 0x80); 0 for s == 0;
+ *   - GEMM: for every 128-wide contraction slab the tensor cores form an
+ *     FP32 partial sum of code products, which is multiplied by the two
+ *     scales of that slab and added to an FP32 accumulator ("promotion" at
+ *     every slab); the result is rounded to BF16 (round-to-nearest-even).
+ *
+ * Layout conventions (every array dense and row-major: element [i][j] of an
+ * [R, C] array is at i*C + j):
+ *   activation, row-wise groups : codes u8 [rows, cols],
+ *                                 scales f32 [cols/128, rows]
+ *   activation, along-token groups (groups of 128 consecutive rows in each
+ *   column, output transposed so tokens are contiguous):
+ *                                 codes u8 [cols, rows],
+ *                                 scales f32 [rows/128, cols]
+ *   weight [n, k]               : codes u8 [n, k], optional transposed
+ *                                 codes u8 [k, n], scales f32 [n/128, k/128]
+ *   bf16 tensors are passed as pointers to 16-bit bfloat16 storage.
+ *
+ * Ownership and streams: the caller allocates and frees every buffer (device
+ * memory unless stated).  No entry point allocates, frees, synchronizes or
+ * keeps a pointer after it returns; all work is enqueued on `stream` (a
+ * cudaStream_t passed as void*; NULL means the legacy default stream) on the
+ * current CUDA device.  Outputs must not overlap inputs.
+ *
+ * Errors: arguments are checked on the host before anything is enqueued; a
+ * failed check returns its status and enqueues nothing.  FP8_ERR_CUDA
+ * reports a failed launch (cudaGetLastError after the launch).  Faults that
+ * happen later on the device surface at the caller's next synchronization,
+ * as with any CUDA work.  Every wait inside a kernel is bounded in time; a
+ * wait that runs out makes the kernel record FP8_ERR_TIMEOUT in a sticky
+ * per-device error word (read it with fp8_get_error) and return without
+ * completing its output.
+ */
+#ifndef FP8BLK_H
+#define FP8BLK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8_OK = 0,
+    FP8_ERR_NULL = 1,     /* a required pointer is NULL                          */
+    FP8_ERR_SHAPE = 2,    /* a size is negative, too large, or not a multiple of
+                             128 where one is required                           */
+    FP8_ERR_ALIGN = 3,    /* a pointer is not 16-byte aligned                     */
+    FP8_ERR_MODE = 4,     /* an unknown mode value                                */
+    FP8_ERR_CUDA = 5,     /* a CUDA runtime call or kernel launch failed          */
+    FP8_ERR_TIMEOUT = 6   /* a bounded wait inside a kernel ran out (sticky)      */
+} fp8_status;
+
+/* Modes of fp8_quantize_act_1x128 (bit flags). */
+enum {
+    FP8_ROWWISE = 1,      /* groups along each row                     */
+    FP8_COLWISE = 2,      /* groups along each column, transposed out  */
+    FP8_BOTH = 3          /* both, from one read of the input          */
+};
+
+/* Largest contraction length (K of fprop, N of dgrad) the fprop/dgrad GEMMs
+ * accept: 256 slabs of 128. */
+#define FP8_MAX_CONTRACTION_FPROP 32768
+
+/*
+ * Activation quantizer, 1x128 groups (row-wise) and/or 128x1 groups along
+ * tokens (column-wise).  Row-wise groups serve fprop (X) and dgrad (dY);
+ * column-wise groups serve wgrad, which contracts over tokens.
+ *
+ *   x_bf16  [rows, cols] bf16, 16-byte aligned.
+ *   rows    >= 0; a multiple of 128 when mode includes FP8_COLWISE.
+ *   cols    >= 0, a multiple of 128.
+ *   mode    FP8_ROWWISE, FP8_COLWISE or FP8_BOTH.
+ *   q_row   [rows, cols] u8 codes; s_row [cols/128, rows] f32 scales
+ *           (written when mode & FP8_ROWWISE; may be NULL otherwise).
+ *   q_colT  [cols, rows] u8 codes; s_col [rows/128, cols] f32 scales
+ *           (written when mode & FP8_COLWISE; may be NULL otherwise).
+ * All pointers used are 16-byte aligned.  rows == 0 or cols == 0 is a no-op
+ * (pointers may then be NULL).
+ */
+fp8_status fp8_quantize_act_1x128(const void *x_bf16, int64_t rows, int64_t cols,
+                                  int mode, uint8_t *q_row, float *s_row,
+                                  uint8_t *q_colT, float *s_col, void *stream);
+
+/*
+ * Weight quantizer, 128x128 blocks.
+ *
+ *   w_bf16  [n, k] bf16, 16-byte aligned; n, k >= 0, multiples of 128.
+ *   wq      [n, k] u8 codes.
+ *   sw      [n/128, k/128] f32 block scales.
+ *   wqT     [k, n] u8 transposed codes (the same bytes: a 128x128 block's
+ *           scale does not depend on orientation), for dgrad; may be NULL.
+ * n == 0 or k == 0 is a no-op (pointers may then be NULL).
+ */
+fp8_status fp8_quantize_weight_128x128(const void *w_bf16, int64_t n, int64_t k,
+                                       uint8_t *wq, float *sw, uint8_t *wqT,
+                                       void *stream);
+
+/*
+ * fprop: Y[m, n] = sum_k X[m, k] W[n, k]   (Y = X W^T), BF16 out.
+ *
+ *   xq [M, K] u8, sx [K/128, M] f32   - row-wise quantized X
+ *   wq [N, K] u8, sw [N/128, K/128] f32 - 128x128 quantized W
+ *   y_bf16 [M, N]
+ *   M >= 0, a multiple of 128; N > 0 and K > 0, multiples of 128;
+ *   K <= FP8_MAX_CONTRACTION_FPROP.  M == 0 is a no-op (pointers may then
+ *   be NULL).
+ */
+fp8_status fp8_block_gemm_fprop(const uint8_t *xq, const float *sx, const uint8_t *wq,
+                                const float *sw, void *y_bf16, int64_t M, int64_t N,
+                                int64_t K, void *stream);
+
+/*
+ * dgrad: dX[m, k] = sum_n dY[m, n] W[n, k]   (dX = dY W), BF16 out.
+ *
+ *   dyq [M, N] u8, sdy [N/128, M] f32 - row-wise quantized dY (groups run
+ *                                        along n, the contraction)
+ *   wqT [K, N] u8                      - transposed weight codes from
+ *                                        fp8_quantize_weight_128x128
+ *   sw  [N/128, K/128] f32             - the weight's block scales (the
+ *                                        same array fprop uses)
+ *   dx_bf16 [M, K]
+ *   M >= 0, a multiple of 128; N > 0 and K > 0, multiples of 128;
+ *   N <= FP8_MAX_CONTRACTION_FPROP.  M == 0 is a no-op (pointers may then
+ *   be NULL).
+ */
+fp8_status fp8_block_gemm_dgrad(const uint8_t *dyq, const float *sdy, const uint8_t *wqT,
+                                const float *sw, void *dx_bf16, int64_t M, int64_t N,
+                                int64_t K, void *stream);
+
+/*
+ * wgrad: dW[n, k] = sum_m dY[m, n] X[m, k]   (dW = dY^T X), contracting over
+ * the M tokens, BF16 out.
+ *
+ *   dyqT [N, M] u8, sdyT [M/128, N] f32 - column-wise (along-token) dY
+ *   xqT  [K, M] u8, sxT  [M/128, K] f32 - column-wise (along-token) X
+ *   dw_bf16 [N, K]
+ *   M > 0, N > 0, K > 0, all multiples of 128.
+ */
+fp8_status fp8_block_gemm_wgrad(const uint8_t *dyqT, const float *sdyT, const uint8_t *xqT,
+                                const float *sxT, void *dw_bf16, int64_t N, int64_t K,
+                                int64_t M, void *stream);
+
+/* Sticky per-device error word: FP8_OK, or the first FP8_ERR_TIMEOUT a
+ * kernel recorded on the current device since the last clear.  Reading it
+ * synchronizes the device. */
+fp8_status fp8_get_error(void);
+fp8_status fp8_clear_error(void);
+
+/* Time limit of every bounded wait inside the kernels launched after this
+ * call, in nanoseconds (default 2e9; 0 restores the default).  Host-side
+ * setting, shared by all devices and threads. */
+fp8_status fp8_set_wait_timeout_ns(uint64_t ns);
+
+/* Text for a status value (static storage). */
+const char *fp8_status_string(fp8_status status);
+
+/* Text of the last CUDA failure behind an FP8_ERR_CUDA returned to the
+ * calling thread ("" if none): the failing call and CUDA's message.  The
+ * storage is per thread and overwritten by the next failure. */
+const char *fp8_last_cuda_error(void);
+
+/* ----------------------------------------------------------- test support */
+
+/* q[i] = E4M3FN(x[i] / scale) with the device rounding path the quantizers
+ * use (IEEE float32 division, then round-to-nearest-even with saturation),
+ * or 0 when scale == 0.  x: n f32 values; q: n bytes; n >= 0. */
+fp8_status fp8_cast_e4m3_scaled(const float *x, float scale, uint8_t *q, int64_t n,
+                                void *stream);
+
+/* Launches one block whose only wait is on a barrier that nothing completes,
+ * so that the bounded wait runs out after the current time limit and
+ * records FP8_ERR_TIMEOUT in the sticky error word.  For testing the timeout
+ * path; nothing else is touched. */
+fp8_status fp8_selftest_wait_timeout(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BLK_H */

@@ -1,0 +1,148 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the
+C ABI, run the oracle on the same seeded inputs, compare.
+
+Acceptance: codes and scales bit-exact; every GEMM output element within
+|gpu - oracle| <= 2e-3 * S + 1e-6, S = sum over slabs of
+|s_a s_b| * sum |a_k||b_k| (the oracle's bound).
+
+The GEMM's output is BF16, and rounding a value y to BF16 (round-to-
+nearest-even, 8 significant bits) moves it by up to 2^-8 |y|.  On the
+Qwen3-1.7B configurations |y| / S stays far below 0.5 and the bound above is
+applied as stated.  The synthetic edge shapes (a contraction of one to three
+slabs in which one x30 outlier channel carries most of every dot product)
+reach |y| / S ~ 0.7, where the correctly rounded BF16 result itself can sit
+further than 2e-3 * S from the exact value; those tests pass
+output_rounding=True, which adds the 2^-8 |y| rounding term."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import blockwise_fp8_pretraining_b200 as fp8
+import oracle
+from blockwise_fp8_pretraining_b200 import synthetic as syn
+
+REL_TOL = 2e-3
+ABS_TOL = 1e-6
+
+
+def dev():
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def assert_bits_equal(gpu: torch.Tensor, ref: np.ndarray, what: str):
+    g = to_np(gpu)
+    if g.dtype == np.float32:
+        g, ref = g.view(np.uint32), np.ascontiguousarray(ref, np.float32).view(np.uint32)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    bad = np.nonzero(g != ref)
+    assert bad[0].size == 0, f"{what}: {bad[0].size} mismatches, first at {tuple(int(b[0]) for b in bad)}"
+
+
+BF16_HALF_ULP_REL = 2.0 ** -8
+
+
+def assert_within_bound(gpu_rows: torch.Tensor, ref: np.ndarray, bound: np.ndarray, what: str,
+                        output_rounding: bool = False):
+    g = to_np(gpu_rows.float()).astype(np.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    lim = REL_TOL * bound + ABS_TOL
+    if output_rounding:
+        lim = lim + BF16_HALF_ULP_REL * np.abs(ref)
+    ok = err <= lim
+    if not np.all(ok):
+        i = np.unravel_index(np.argmax(err / lim), err.shape)
+        raise AssertionError(f"{what}: {int((~ok).sum())} elements outside the bound; worst at {i}: "
+                             f"gpu={g[i]!r} oracle={ref[i]!r} S={bound[i]!r}")
+
+
+# ----------------------------------------------------------------- quantizers
+
+def check_act(x: torch.Tensor, mode=fp8.BOTH):
+    """Quantize x (CPU bf16) on the GPU in `mode` and compare bit-exactly
+    with the oracle.  Returns the GPU outputs."""
+    xb = syn.bf16_bits(x)
+    q_row, s_row, q_colT, s_col = fp8.fp8_quantize_act_1x128(x.to(dev()), mode)
+    torch.cuda.synchronize()
+    if mode & fp8.ROWWISE:
+        q_o, s_o = oracle.quantize_act_rowwise(xb)
+        assert_bits_equal(q_row, q_o, "row-wise codes")
+        assert_bits_equal(s_row, s_o, "row-wise scales")
+    if mode & fp8.COLWISE:
+        q_o, s_o = oracle.quantize_act_colwise(xb)
+        assert_bits_equal(q_colT, q_o, "column-wise codes")
+        assert_bits_equal(s_col, s_o, "column-wise scales")
+    return q_row, s_row, q_colT, s_col
+
+
+def check_weight(w: torch.Tensor):
+    wq, sw, wqT = fp8.fp8_quantize_weight_128x128(w.to(dev()))
+    torch.cuda.synchronize()
+    q_o, s_o = oracle.quantize_weight(syn.bf16_bits(w))
+    assert_bits_equal(wq, q_o, "weight codes")
+    assert_bits_equal(sw, s_o, "weight scales")
+    assert_bits_equal(wqT, np.ascontiguousarray(q_o.T), "transposed weight codes")
+    return wq, sw, wqT
+
+
+# ---------------------------------------------------------------------- GEMMs
+
+def pick_rows(total: int, count: int, seed: int) -> np.ndarray:
+    """Seeded sample of output rows that always includes the first and last
+    row of the first and last 128-row tile."""
+    if count >= total:
+        return np.arange(total)
+    rng = np.random.default_rng(seed)
+    fixed = np.array(sorted({0, min(127, total - 1), max(0, total - 128), total - 1}))
+    rest = rng.choice(total, size=max(0, count - fixed.size), replace=False)
+    return np.unique(np.concatenate([fixed, rest]))
+
+
+def check_fprop(x: torch.Tensor, w: torch.Tensor, rows=None, what="fprop", output_rounding=False):
+    """GPU: quantize + fprop through the C ABI; oracle: quantize + fprop on
+    the selected rows (all when rows is None).  Returns the GPU output."""
+    d = dev()
+    xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x.to(d), fp8.ROWWISE)
+    wq, sw, _ = fp8.fp8_quantize_weight_128x128(w.to(d), transposed=False)
+    y = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+    torch.cuda.synchronize()
+    xq_o, sx_o = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    wq_o, sw_o = oracle.quantize_weight(syn.bf16_bits(w))
+    y_o, b_o = oracle.gemm_fprop(xq_o, sx_o, wq_o, sw_o, rows=rows)
+    sel = y if rows is None else y[torch.as_tensor(rows, device=d)]
+    assert_within_bound(sel, y_o, b_o, what, output_rounding)
+    return y
+
+
+def check_dgrad(dy: torch.Tensor, w: torch.Tensor, rows=None, what="dgrad", output_rounding=False):
+    d = dev()
+    dyq, sdy, _, _ = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.ROWWISE)
+    _, sw, wqT = fp8.fp8_quantize_weight_128x128(w.to(d))
+    dx = fp8.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw)
+    torch.cuda.synchronize()
+    dyq_o, sdy_o = oracle.quantize_act_rowwise(syn.bf16_bits(dy))
+    wq_o, sw_o = oracle.quantize_weight(syn.bf16_bits(w))
+    dx_o, b_o = oracle.gemm_dgrad(dyq_o, sdy_o, wq_o, sw_o, rows=rows)
+    sel = dx if rows is None else dx[torch.as_tensor(rows, device=d)]
+    assert_within_bound(sel, dx_o, b_o, what, output_rounding)
+    return dx
+
+
+def check_wgrad(dy: torch.Tensor, x: torch.Tensor, rows=None, what="wgrad", output_rounding=False):
+    d = dev()
+    _, _, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.COLWISE)
+    _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
+    dw = fp8.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT)
+    torch.cuda.synchronize()
+    dyqT_o, sdyT_o = oracle.quantize_act_colwise(syn.bf16_bits(dy))
+    xqT_o, sxT_o = oracle.quantize_act_colwise(syn.bf16_bits(x))
+    dw_o, b_o = oracle.gemm_wgrad(dyqT_o, sdyT_o, xqT_o, sxT_o, rows=rows)
+    sel = dw if rows is None else dw[torch.as_tensor(rows, device=d)]
+    assert_within_bound(sel, dw_o, b_o, what, output_rounding)
+    return dw

@@ -1,0 +1,114 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+the header declares, and rejects bad arguments on the host before touching
+the device (so the fake pointers below are never dereferenced)."""
+import ctypes
+
+import pytest
+
+import blockwise_fp8_pretraining_b200 as fp8
+from blockwise_fp8_pretraining_b200 import _abi
+
+OK, NULL, SHAPE, ALIGN, MODE = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from blockwise_fp8_pretraining_b200 import build
+
+    build.build()
+    return fp8.load()
+
+
+def test_header_declares_the_expected_entry_points():
+    names = set(fp8.header_functions())
+    for want in ("fp8_quantize_act_1x128", "fp8_quantize_weight_128x128", "fp8_block_gemm_fprop",
+                 "fp8_block_gemm_dgrad", "fp8_block_gemm_wgrad", "fp8_get_error",
+                 "fp8_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_header_function(lib):
+    for name in fp8.header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_python_binding_has_every_header_function():
+    for name in fp8.header_functions():
+        assert hasattr(fp8, name), name
+
+
+def test_status_strings(lib):
+    for st in range(7):
+        assert lib.fp8_status_string(st)
+    assert fp8.fp8_status_string(99) == "unknown status"
+
+
+A16 = 0x10000          # fake, 16-byte aligned, never dereferenced
+MIS = 0x10008          # fake, misaligned
+S = ctypes.c_void_p(0)
+
+
+def P(v):
+    return ctypes.c_void_p(v)
+
+
+def test_quantize_act_rejections(lib):
+    q = lib.fp8_quantize_act_1x128
+    assert q(P(A16), 256, 2048, 0, P(A16), P(A16), P(A16), P(A16), S) == MODE
+    assert q(P(A16), 256, 2048, 5, P(A16), P(A16), P(A16), P(A16), S) == MODE
+    assert q(P(A16), 256, 100, 1, P(A16), P(A16), None, None, S) == SHAPE
+    assert q(P(A16), -1, 128, 1, P(A16), P(A16), None, None, S) == SHAPE
+    assert q(P(A16), 100, 128, 2, None, None, P(A16), P(A16), S) == SHAPE   # colwise needs rows%128
+    assert q(None, 256, 128, 1, P(A16), P(A16), None, None, S) == NULL
+    assert q(P(A16), 256, 128, 1, None, P(A16), None, None, S) == NULL
+    assert q(P(A16), 256, 128, 3, P(A16), P(A16), None, P(A16), S) == NULL
+    assert q(P(MIS), 256, 128, 1, P(A16), P(A16), None, None, S) == ALIGN
+    assert q(P(A16), 256, 128, 2, None, None, P(A16), P(MIS), S) == ALIGN
+    # empty inputs are a no-op that launches nothing
+    assert q(P(A16), 0, 128, 3, P(A16), P(A16), P(A16), P(A16), S) == OK
+    assert q(P(A16), 5, 0, 1, P(A16), P(A16), None, None, S) == OK
+
+
+def test_quantize_weight_rejections(lib):
+    q = lib.fp8_quantize_weight_128x128
+    assert q(P(A16), 100, 128, P(A16), P(A16), None, S) == SHAPE
+    assert q(P(A16), 128, 129, P(A16), P(A16), None, S) == SHAPE
+    assert q(P(A16), 128, 128, None, P(A16), None, S) == NULL
+    assert q(P(A16), 128, 128, P(A16), P(A16), P(MIS), S) == ALIGN
+    assert q(P(A16), 0, 128, P(A16), P(A16), None, S) == OK
+
+
+@pytest.mark.parametrize("name", ["fp8_block_gemm_fprop", "fp8_block_gemm_dgrad"])
+def test_fprop_dgrad_rejections(lib, name):
+    g = getattr(lib, name)
+    a = [P(A16)] * 5
+    assert g(*a, 100, 256, 256, S) == SHAPE          # M not a multiple of 128
+    assert g(*a, 128, 0, 256, S) == SHAPE
+    assert g(*a, 128, 256, 0, S) == SHAPE
+    assert g(*a, 128, 200, 256, S) == SHAPE
+    big = fp8.MAX_CONTRACTION_FPROP + 128
+    if name == "fp8_block_gemm_fprop":
+        assert g(*a, 128, 256, big, S) == SHAPE
+    else:
+        assert g(*a, 128, big, 256, S) == SHAPE
+    assert g(None, *a[1:], 128, 256, 256, S) == NULL
+    assert g(*a[:4], None, 128, 256, 256, S) == NULL
+    assert g(*a[:2], P(MIS), *a[3:], 128, 256, 256, S) == ALIGN
+    assert g(*a, 0, 256, 256, S) == OK               # M == 0: nothing to do
+
+
+def test_wgrad_rejections(lib):
+    g = lib.fp8_block_gemm_wgrad
+    a = [P(A16)] * 5
+    assert g(*a, 256, 256, 0, S) == SHAPE            # no tokens
+    assert g(*a, 256, 256, 100, S) == SHAPE
+    assert g(*a, 200, 256, 256, S) == SHAPE
+    assert g(*a[:3], None, a[4], 256, 256, 256, S) == NULL
+    assert g(*a[:4], P(MIS), 256, 256, 256, S) == ALIGN
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(_abi._build, "LIB", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_abi, "_lib", None)
+    with pytest.raises(OSError):
+        _abi.load()

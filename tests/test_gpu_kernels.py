@@ -1,0 +1,225 @@
+"""GPU parity of every kernel against the CPU oracle at sizes the oracle
+finishes in seconds: several tiles, ragged tails (row counts that are not a
+multiple of a block's rows, N = 128 * odd against 256-wide GEMM tiles, grids
+with fewer tiles than SMs and with a partial last wave), heavy tails, zero
+groups, and the degenerate cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+import blockwise_fp8_pretraining_b200 as fp8
+import oracle
+from blockwise_fp8_pretraining_b200 import synthetic as syn
+
+from _parity import (assert_bits_equal, check_act, check_dgrad, check_fprop, check_wgrad,
+                     check_weight, dev, pick_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fp8.load()
+    fp8.fp8_clear_error()
+    yield
+    assert fp8.fp8_get_error() == 0
+
+
+# ------------------------------------------------------------- element cast
+
+def test_cast_matches_oracle_on_grid_midpoints_and_saturation():
+    pos = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mid = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    vals = np.concatenate([
+        pos.astype(np.float32), mid, np.nextafter(mid, np.float32(0)),
+        np.nextafter(mid, np.float32(np.inf)),
+        np.array([448, 463.99, 464, 470, 480, 1e4, 1e30, 3e38, 0.0, 1e-30, 1e-45], np.float32),
+    ])
+    vals = np.concatenate([vals, -vals]).astype(np.float32)
+    for scale in (1.0, 0.5, 2.0 ** -20, 3.0, 1e-3, 7.0 / 448.0):
+        q = fp8.fp8_cast_e4m3_scaled(torch.from_numpy(vals).to(dev()), scale)
+        ref = oracle.e4m3_encode((vals / np.float32(scale)).astype(np.float32))
+        assert_bits_equal(q, ref, f"cast scale={scale}")
+    q0 = fp8.fp8_cast_e4m3_scaled(torch.from_numpy(vals).to(dev()), 0.0)
+    assert torch.all(q0 == 0)
+
+
+def test_cast_random_fp32_sweep():
+    rng = np.random.default_rng(5)
+    v = (np.exp(rng.uniform(np.log(1e-12), np.log(1e6), 2_000_000))
+         * np.where(rng.random(2_000_000) < 0.5, -1, 1)).astype(np.float32)
+    for scale in (1.0, 0.013, 1e-7):
+        q = fp8.fp8_cast_e4m3_scaled(torch.from_numpy(v).to(dev()), scale)
+        assert_bits_equal(q, oracle.e4m3_encode((v / np.float32(scale)).astype(np.float32)),
+                          f"random cast {scale}")
+
+
+# ------------------------------------------------------------- quantizers
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (3, 384), (127, 256), (129, 2048), (1000, 640),
+                                       (256, 2048)])
+def test_rowwise_ragged_rows(rows, cols):
+    x = syn.activation_bf16(rows, cols, max(1, cols // 100), 30.0, syn.generator(rows + cols))
+    check_act(x, fp8.ROWWISE)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (384, 2048), (1024, 640)])
+@pytest.mark.parametrize("mode", [fp8.COLWISE, fp8.BOTH])
+def test_colwise_and_dual(rows, cols, mode):
+    x = syn.activation_bf16(rows, cols, max(1, cols // 100), 30.0, syn.generator(rows * 3 + cols))
+    check_act(x, mode)
+
+
+def test_quantizers_heavy_tail_zero_and_negative_zero_groups():
+    x = syn.student_t_bf16((512, 1024), seed=11).float()
+    x[5, :] = 0.0                     # all-zero row groups
+    x[6, :] = -0.0                    # groups of negative zeros
+    x[:, 128:256] = 0.0               # all-zero column block
+    x[7, 300] = 3.0e38                # near the top of the bf16 range
+    x[8, 0:128] = 1e-40               # bf16 subnormals, scale becomes subnormal
+    x[9, 0] = -1e-40
+    x = x.to(torch.bfloat16)
+    check_act(x, fp8.BOTH)
+    check_act(x, fp8.ROWWISE)
+    check_act(x, fp8.COLWISE)
+
+
+@pytest.mark.parametrize("n,k", [(128, 128), (384, 256), (2048, 2048), (256, 6144)])
+def test_weight_blocks(n, k):
+    w = syn.normal_bf16((n, k), 0.02, syn.generator(n + k))
+    check_weight(w)
+
+
+def test_weight_without_transposed_copy_and_special_blocks():
+    w = syn.normal_bf16((256, 384), 0.02, syn.generator(3)).float()
+    w[:128, :128] = 0.0
+    w[128:, 256:] = -0.0
+    w = w.to(torch.bfloat16)
+    wq, sw, wqT = fp8.fp8_quantize_weight_128x128(w.to(dev()), transposed=False)
+    assert wqT is None
+    q_o, s_o = oracle.quantize_weight(syn.bf16_bits(w))
+    assert_bits_equal(wq, q_o, "codes")
+    assert_bits_equal(sw, s_o, "scales")
+
+
+# ------------------------------------------------------------------ GEMMs
+
+GEMM_SHAPES = [
+    (128, 128, 128),      # one tile, one slab
+    (128, 384, 256),      # ragged N: one full and one half-width tile
+    (256, 640, 512),
+    (384, 256, 1152),     # odd number of slabs
+    (1280, 2304, 384),    # 90 tiles: fewer tiles than SMs
+    (4096, 2560, 256),    # 320 tiles: partial last wave
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_fprop_small(M, N, K):
+    g = syn.generator(M + N + K)
+    x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
+    w = syn.normal_bf16((N, K), 0.02, g)
+    rows = None if M <= 384 else pick_rows(M, 96, M)
+    check_fprop(x, w, rows, output_rounding=True)
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_dgrad_small(M, N, K):
+    # dX [M, K] = dY [M, N] W [N, K]
+    g = syn.generator(M * 7 + N + K)
+    dy = syn.normal_bf16((M, N), 1e-3, g)
+    w = syn.normal_bf16((N, K), 0.02, g)
+    rows = None if M <= 384 else pick_rows(M, 96, M)
+    check_dgrad(dy, w, rows, output_rounding=True)
+
+
+@pytest.mark.parametrize("N,K,M", [(128, 128, 128), (384, 256, 256), (256, 640, 384),
+                                   (1280, 2304, 256), (2560, 4096, 128)])
+def test_wgrad_small(N, K, M):
+    g = syn.generator(N * 5 + K + M)
+    dy = syn.normal_bf16((M, N), 1e-3, g)
+    x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
+    rows = None if N <= 384 else pick_rows(N, 96, N)
+    check_wgrad(dy, x, rows, output_rounding=True)
+
+
+def test_tiny_config_fprop_dgrad_wgrad_full():
+    """X [256, 2048] (4 channels x50), W [2048, 2048], dY [256, 2048]: every
+    output element of the three GEMMs against the oracle."""
+    c = syn.tiny(seed=0)
+    check_act(c["x"], fp8.BOTH)
+    check_act(c["dy"], fp8.BOTH)
+    check_weight(c["w"])
+    check_fprop(c["x"], c["w"])
+    check_dgrad(c["dy"], c["w"])
+    check_wgrad(c["dy"], c["x"], rows=pick_rows(2048, 256, 1))
+
+
+def test_gemm_degenerate_inputs():
+    """All-zero operands give exact zeros; all-ones give the closed form."""
+    d = dev()
+    z = torch.zeros((256, 512), dtype=torch.bfloat16)
+    w = syn.normal_bf16((384, 512), 0.02, syn.generator(9))
+    y = check_fprop(z, w)
+    assert torch.all(y == 0)
+    ones = torch.ones((128, 128), dtype=torch.bfloat16)
+    y = check_fprop(ones, ones, output_rounding=True)
+    s = float(np.float32(1.0) / np.float32(448.0))
+    want = torch.tensor(128 * (448 * s) ** 2, dtype=torch.float32).to(torch.bfloat16)
+    assert torch.all(y.cpu() == want)
+
+
+def test_empty_inputs_are_noops():
+    d = dev()
+    xq = torch.empty((0, 256), dtype=torch.uint8, device=d)
+    sx = torch.empty((2, 0), dtype=torch.float32, device=d)
+    wq = torch.zeros((128, 256), dtype=torch.uint8, device=d)
+    sw = torch.zeros((1, 2), dtype=torch.float32, device=d)
+    y = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+    assert y.shape == (0, 128)
+    wqT = torch.zeros((256, 128), dtype=torch.uint8, device=d)
+    dx = fp8.fp8_block_gemm_dgrad(torch.empty((0, 128), dtype=torch.uint8, device=d),
+                                  torch.empty((1, 0), dtype=torch.float32, device=d), wqT,
+                                  torch.zeros((1, 2), dtype=torch.float32, device=d))
+    assert dx.shape == (0, 256)
+    q_row, s_row, q_colT, s_col = fp8.fp8_quantize_act_1x128(
+        torch.empty((0, 256), dtype=torch.bfloat16, device=d), fp8.BOTH)
+    assert q_row.shape == (0, 256) and s_col.shape == (0, 256)
+    wq0, sw0, wqT0 = fp8.fp8_quantize_weight_128x128(torch.empty((0, 128), dtype=torch.bfloat16, device=d))
+    assert wq0.shape == (0, 128) and wqT0.shape == (128, 0)
+    torch.cuda.synchronize()
+
+
+def test_outputs_do_not_depend_on_stream_or_repeat():
+    """Same inputs on another stream and a second run give identical bits
+    (each output element is produced by one thread in a fixed order)."""
+    c = syn.tiny(seed=3)
+    d = dev()
+    x, w = c["x"].to(d), c["w"].to(d)
+    xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x, fp8.ROWWISE)
+    wq, sw, _ = fp8.fp8_quantize_weight_128x128(w, transposed=False)
+    y1 = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y2 = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+# --------------------------------------------------------------- time-outs
+
+def test_bounded_wait_times_out_and_reports():
+    fp8.fp8_clear_error()
+    fp8.fp8_set_wait_timeout_ns(2_000_000)          # 2 ms
+    try:
+        fp8.fp8_selftest_wait_timeout()
+        assert fp8.fp8_get_error() == 6              # FP8_ERR_TIMEOUT
+    finally:
+        fp8.fp8_set_wait_timeout_ns(0)
+        fp8.fp8_clear_error()
+    # the context is still usable afterwards
+    check_fprop(syn.normal_bf16((128, 128), 1.0, syn.generator(1)),
+                syn.normal_bf16((128, 128), 0.02, syn.generator(2)))
