@@ -20,6 +20,7 @@ from ._abi import (  # noqa: F401
     fp8_last_cuda_error,
     fp8_quantize_act_1x128,
     fp8_quantize_weight_128x128,
+    fp8_selftest_division,
     fp8_selftest_wait_timeout,
     fp8_set_wait_timeout_ns,
     fp8_status_string,

@@ -64,6 +64,7 @@ def load() -> ctypes.CDLL:
         "fp8_set_wait_timeout_ns": [ctypes.c_uint64],
         "fp8_cast_e4m3_scaled": [p, ctypes.c_float, p, i64, p],
         "fp8_selftest_wait_timeout": [p],
+        "fp8_selftest_division": [p, p],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -248,6 +249,16 @@ def fp8_cast_e4m3_scaled(x, scale: float, q=None, stream=None):
     _check(lib.fp8_cast_e4m3_scaled(_ptr(x), ctypes.c_float(scale), _ptr(q), n, _stream(stream)),
            "fp8_cast_e4m3_scaled")
     return q
+
+
+def fp8_selftest_division(stream=None):
+    """Returns (code mismatches, first code mismatch, quotient-bit
+    mismatches with |x/s| >= 2^-12, first such, quotient-bit mismatches
+    below 2^-12)."""
+    res = torch.zeros(6, dtype=torch.int64, device="cuda")
+    _check(load().fp8_selftest_division(_ptr(res), _stream(stream)), "fp8_selftest_division")
+    torch.cuda.synchronize()
+    return tuple(res.cpu().tolist()[:5])
 
 
 def fp8_selftest_wait_timeout(stream=None) -> None:

@@ -99,6 +99,25 @@ fp8_status make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows,
     return FP8_OK;
 }
 
+// Row-major [rows, cols] bf16 output, boxes of 32 rows x 64 columns (128
+// bytes) in the 128-byte swizzle the epilogue's staging buffers use.
+fp8_status make_output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return FP8_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64u, 32u};
+    cuuint32_t estride[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled(output): CUresult %d", static_cast<int>(r));
+        return FP8_ERR_CUDA;
+    }
+    return FP8_OK;
+}
+
 // Shared launcher of the three GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
 // codes, both K-major; scales described by `p`.
 template <int SCALE>
@@ -117,16 +136,17 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, gemm::Params p, cudaS
         g_gemm_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
     }
 
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mc;
     if ((st = make_operand_map(&ma, a, p.M, p.K, gemm::BM)) != FP8_OK) return st;
     if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN)) != FP8_OK) return st;
+    if ((st = make_output_map(&mc, p.out, p.M, p.N)) != FP8_OK) return st;
 
     p.tiles_m = static_cast<int>((p.M + gemm::BM - 1) / gemm::BM);
     p.tiles_n = static_cast<int>((p.N + gemm::BN - 1) / gemm::BN);
     p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    gemm::gemm_kernel<SCALE><<<grid, gemm::THREADS, gemm::SMEM_BYTES, stream>>>(ma, mb, p);
+    gemm::gemm_kernel<SCALE><<<grid, gemm::THREADS, gemm::SMEM_BYTES, stream>>>(ma, mb, mc, p);
     return last_launch_status("gemm launch");
 }
 
@@ -309,6 +329,13 @@ fp8_status fp8_cast_e4m3_scaled(const float* x, float scale, uint8_t* q, int64_t
     cast_e4m3_scaled_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         x, scale, q, n);
     return last_launch_status("cast launch");
+}
+
+fp8_status fp8_selftest_division(unsigned long long* result, void* stream) {
+    if (!result) return FP8_ERR_NULL;
+    if (!aligned16(result)) return FP8_ERR_ALIGN;
+    division_selftest_kernel<<<0x7F7F, 256, 0, static_cast<cudaStream_t>(stream)>>>(result);
+    return last_launch_status("division self-test launch");
 }
 
 fp8_status fp8_selftest_wait_timeout(void* stream) {

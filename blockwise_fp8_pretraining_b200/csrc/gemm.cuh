@@ -21,10 +21,13 @@
 //   warps 2, 3  idle (they complete warpgroup 0, which gives registers away)
 //   warps 4..11 promotion + epilogue: each thread owns one output row (TMEM
 //               lane) and 128 columns, pulls the slab partials with
-//               tcgen05.ld, does acc = fma(s_a * s_b, P, acc) in registers,
-//               releases the TMEM buffer, and after the last slab rounds to
-//               BF16 and stores.  TMEM double buffering lets promotion of
-//               slab t overlap the MMAs of slab t+1.
+//               tcgen05.ld (two 32-column loads per wait), releases the TMEM
+//               buffer as soon as the last load has landed, and does
+//               acc = fma(s_a * s_b, P, acc) in registers with packed FP32x2
+//               FMAs.  After the last slab it rounds to BF16 into a per-warp
+//               128-byte-swizzled staging buffer that TMA stores to global
+//               memory asynchronously.  TMEM double buffering lets promotion
+//               of slab t overlap the MMAs of slab t+1.
 // Scale modes:
 //   kScaleRowBlock (fprop, dgrad): s_a is per output row (1x128 activation
 //     groups), s_b per 128-column block of the weight (128x128 blocks), so
@@ -47,7 +50,7 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;              // one quantization slab
 constexpr int UMMA_K = 32;           // K of one kind::f8f6f4 MMA
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int SSTAGES = 8;
 constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
@@ -68,12 +71,17 @@ constexpr int SCALE_SLOT_BYTES = (BM + BN) * 4;
 constexpr int MAX_KB = 256;          // slabs of a fprop/dgrad contraction
 constexpr int SB_REGS = MAX_KB / 32;
 
+constexpr int OUT_WARP_BYTES = 32 * 128 * 2;     // 32 rows x 128 BF16 per epilogue warp
+
 constexpr int OFF_SCALES = STAGES * STAGE_BYTES;
-constexpr int OFF_BARS = OFF_SCALES + SSTAGES * SCALE_SLOT_BYTES;
+constexpr int OFF_OUT = OFF_SCALES + SSTAGES * SCALE_SLOT_BYTES;
+constexpr int OFF_BARS = OFF_OUT + EPI_WARPS * OUT_WARP_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 * SSTAGES + 1;
 constexpr int OFF_TMEM_SLOT = OFF_BARS + NUM_BARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(OFF_OUT % 1024 == 0, "swizzled staging must be 1024-byte aligned");
 
 constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
 
@@ -135,7 +143,7 @@ __device__ __forceinline__ void load_sb(float (&regs)[SB_REGS], const Params& p,
 template <int SCALE>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tmC, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -179,6 +187,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmC);
     }
     tc_fence_before();
     __syncthreads();
@@ -307,47 +316,55 @@ __global__ void __launch_bounds__(THREADS, 1)
                     reinterpret_cast<const float*>(smem + OFF_SCALES + ss * SCALE_SLOT_BYTES);
                 const float sa = slot[row_in_tile];
                 const uint32_t taddr = lane_base + buf * BN + half * 128;
+                float2 cpair = make_float2(0.0f, 0.0f);
                 if (SCALE == kScaleRowBlock) {
                     const float c = sa * pick_sb(sb_cur, kb);
+                    cpair = make_float2(c, c);
+                }
+                const float* sbv = slot + BM + half * 128;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(taddr + ch * 32, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            acc[ch * 32 + j] = fmaf(c, __uint_as_float(r[j]), acc[ch * 32 + j]);
+                for (int g = 0; g < 2; ++g) {
+                    uint32_t r[2][32];
+                    tmem_ld_32x32b_x32(taddr + g * 64, r[0]);
+                    tmem_ld_32x32b_x32(taddr + g * 64 + 32, r[1]);
+                    tmem_ld_wait();
+                    if (g == 1) {
+                        // Both halves of the buffer are in registers: hand it back.
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bars.tempty_(buf));
                     }
-                } else {
-                    const float* sbv = slot + BM + half * 128;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(taddr + ch * 32, r);
-                        tmem_ld_wait();
+                    for (int q = 0; q < 2; ++q) {
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 b4 = *reinterpret_cast<const float4*>(sbv + ch * 32 + j);
-                            acc[ch * 32 + j + 0] = fmaf(sa * b4.x, __uint_as_float(r[j + 0]), acc[ch * 32 + j + 0]);
-                            acc[ch * 32 + j + 1] = fmaf(sa * b4.y, __uint_as_float(r[j + 1]), acc[ch * 32 + j + 1]);
-                            acc[ch * 32 + j + 2] = fmaf(sa * b4.z, __uint_as_float(r[j + 2]), acc[ch * 32 + j + 2]);
-                            acc[ch * 32 + j + 3] = fmaf(sa * b4.w, __uint_as_float(r[j + 3]), acc[ch * 32 + j + 3]);
+                        for (int j = 0; j < 32; j += 2) {
+                            const int a = g * 64 + q * 32 + j;
+                            float2 cc = cpair;
+                            if (SCALE == kScaleOuter) {
+                                const float2 b2 = *reinterpret_cast<const float2*>(sbv + a);
+                                cc = __fmul2_rn(make_float2(sa, sa), b2);
+                            }
+                            const float2 v = __ffma2_rn(
+                                cc, make_float2(__uint_as_float(r[q][j]), __uint_as_float(r[q][j + 1])),
+                                make_float2(acc[a], acc[a + 1]));
+                            acc[a] = v.x;
+                            acc[a + 1] = v.y;
                         }
                     }
                 }
-                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bars.tempty_(buf));
-                    mbar_arrive(bars.sempty_(ss));
-                }
+                if (lane == 0) mbar_arrive(bars.sempty_(ss));
             }
             if (!ok) break;
 
-            // BF16 round-to-nearest-even and store of this thread's row.
+            // BF16 round-to-nearest-even into this warp's staging buffer (two
+            // 32 x 64 boxes, 128-byte rows, 16-byte chunk j of row r at
+            // position j ^ (r % 8)), then TMA stores of the two boxes.
             const int col0 = n0 + half * 128;
             if (col0 < p.N) {
-                __nv_bfloat16* dst = p.out + static_cast<int64_t>(m0 + row_in_tile) * p.N + col0;
+                uint8_t* stage_out = smem + OFF_OUT + ew * OUT_WARP_BYTES;
+                if (lane == 0) bulk_wait_group_read0();     // previous tile's store has read the buffer
+                __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 128; j += 8) {
                     uint4 o;
@@ -359,7 +376,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                     o.y = *reinterpret_cast<uint32_t*>(&h1);
                     o.z = *reinterpret_cast<uint32_t*>(&h2);
                     o.w = *reinterpret_cast<uint32_t*>(&h3);
-                    *reinterpret_cast<uint4*>(dst + j) = o;
+                    const int box = j >> 6;                 // which 64-column box
+                    const int chunk = (j & 63) >> 3;        // 16-byte chunk in the 128-byte row
+                    *reinterpret_cast<uint4*>(stage_out + box * 4096 + lane * 128 +
+                                              ((chunk ^ (lane & 7)) << 4)) = o;
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    const uint32_t src = smem_u32(stage_out);
+                    tma_store_2d(&tmC, src, col0, m0 + quarter * 32);
+                    tma_store_2d(&tmC, src + 4096, col0 + 64, m0 + quarter * 32);
+                    bulk_commit_group();
                 }
             }
             if (SCALE == kScaleRowBlock) {
@@ -367,6 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int r = 0; r < SB_REGS; ++r) sb_cur[r] = sb_next[r];
             }
         }
+        if (lane == 0) bulk_wait_group0();                 // output stores complete
     }
 
     tc_fence_before();

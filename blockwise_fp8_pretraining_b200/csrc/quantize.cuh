@@ -32,17 +32,46 @@ __device__ __forceinline__ float amax8(const uint4& v) {
 
 __device__ __forceinline__ float group_scale(float amax) { return __fdiv_rn(amax, 448.0f); }
 
-// Codes of two values with scale s (s > 0): IEEE division, then E4M3 RNE.
-__device__ __forceinline__ uint32_t code2(float lo, float hi, float s) {
-    return cvt_e4m3x2(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
+// x / s correctly rounded (IEEE float32, round-to-nearest-even) for one
+// divisor s shared by a whole group, without a division per element.
+// Markstein's scheme (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// r = RN(1/s) and q0 = RN(x r), the remainder e = x - s q0 is exact in one
+// FMA and RN(q0 + e r) is the correctly rounded quotient.  The remainder is
+// exact only while it stays a normal float, so divisors outside
+// [2^-100, 2^100] (groups of tiny or huge bf16 values) take the IEEE
+// division instead.  copysign keeps the sign of -0 / s.  An exhaustive GPU
+// check (fp8_selftest_division) compares the E4M3 codes and the quotient
+// bits of both paths for every (bf16 amax, bf16 x) pair a group can hold.
+struct Quotient {
+    float s, r;
+    bool fast;
+    __device__ __forceinline__ explicit Quotient(float s_) : s(s_), r(0.0f) {
+#ifdef __CUDA_ARCH__
+        r = __frcp_rn(s_);
+#endif
+        fast = (s_ >= 0x1p-100f) && (s_ <= 0x1p100f);
+    }
+    __device__ __forceinline__ float operator()(float x) const {
+        if (!fast) return __fdiv_rn(x, s);
+        const float q0 = x * r;
+        const float e = fmaf(-s, q0, x);
+        return copysignf(fmaf(e, r, q0), x);
+    }
+};
+
+// Codes of two values of a group (s > 0): quotient, then E4M3 RNE.
+__device__ __forceinline__ uint32_t code2(float lo, float hi, const Quotient& q) {
+    return cvt_e4m3x2(q(lo), q(hi));
 }
 
 // Codes of the 8 bf16 values of a chunk, packed in memory order.
 __device__ __forceinline__ uint2 encode8(const uint4& v, float s) {
     if (s == 0.0f) return make_uint2(0u, 0u);
+    const Quotient q(s);
     uint2 r;
-    r.x = code2(bf16_lo(v.x), bf16_hi(v.x), s) | (code2(bf16_lo(v.y), bf16_hi(v.y), s) << 16);
-    r.y = code2(bf16_lo(v.z), bf16_hi(v.z), s) | (code2(bf16_lo(v.w), bf16_hi(v.w), s) << 16);
+    r.x = code2(bf16_lo(v.x), bf16_hi(v.x), q) | (code2(bf16_lo(v.y), bf16_hi(v.y), q) << 16);
+    r.y = code2(bf16_lo(v.z), bf16_hi(v.z), q) | (code2(bf16_lo(v.w), bf16_hi(v.w), q) << 16);
     return r;
 }
 
@@ -101,7 +130,7 @@ enum TileMode : int { kTileColwise = 0, kTileBoth = 1, kTileWeight = 2 };
 //   kTileWeight  : q_row = codes [rows, cols], s_col = block scales
 //                  [rows/128, cols/128], q_colT = transposed codes or NULL
 template <int MODE>
-__global__ void __launch_bounds__(256) quant_tile_kernel(const uint4* __restrict__ x,
+__global__ void __launch_bounds__(256, 3) quant_tile_kernel(const uint4* __restrict__ x,
                                                          int64_t rows, int64_t cols,
                                                          uint8_t* __restrict__ q_row,
                                                          float* __restrict__ s_row,
@@ -196,18 +225,19 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(const uint4* __restrict
 
     // Transposed codes: 32 consecutive tokens of columns 2p and 2p+1.
     uint32_t b0[8], b1[8];
+    const Quotient q0(s0), q1(s1);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const uint32_t wa = w[4 * j], wb = w[4 * j + 1], wc = w[4 * j + 2], wd = w[4 * j + 3];
         if (s0 == 0.0f) {
             b0[j] = 0u;
         } else {
-            b0[j] = code2(bf16_lo(wa), bf16_lo(wb), s0) | (code2(bf16_lo(wc), bf16_lo(wd), s0) << 16);
+            b0[j] = code2(bf16_lo(wa), bf16_lo(wb), q0) | (code2(bf16_lo(wc), bf16_lo(wd), q0) << 16);
         }
         if (s1 == 0.0f) {
             b1[j] = 0u;
         } else {
-            b1[j] = code2(bf16_hi(wa), bf16_hi(wb), s1) | (code2(bf16_hi(wc), bf16_hi(wd), s1) << 16);
+            b1[j] = code2(bf16_hi(wa), bf16_hi(wb), q1) | (code2(bf16_hi(wc), bf16_hi(wd), q1) << 16);
         }
     }
     uint8_t* dst0 = q_colT + (c0 + 2 * p) * rows + r0 + qq * 32;
@@ -224,6 +254,42 @@ __global__ void cast_e4m3_scaled_kernel(const float* __restrict__ x, float scale
                                         uint8_t* __restrict__ q, int64_t n) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i < n) q[i] = (scale == 0.0f) ? 0 : static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x[i], scale), 0.0f) & 0xFFu);
+}
+
+// Every positive finite bf16 amax (one block each) against every bf16 x with
+// |x| <= amax: E4M3 code and quotient bits of the group path (Quotient)
+// versus the IEEE division.  result[0] += code mismatches, result[1] = first
+// code mismatch (amax bits << 16 | x bits), result[2] += quotient-bit
+// mismatches with |x / s| >= 2^-12 (where a code can be nonzero), result[3]
+// = first such mismatch, result[4] += quotient-bit mismatches below 2^-12.
+__global__ void __launch_bounds__(256) division_selftest_kernel(unsigned long long* result) {
+    const uint32_t abits = blockIdx.x + 1u;                 // 0x0001 .. 0x7F7F
+    const float amax = __uint_as_float(abits << 16);
+    const float s = group_scale(amax);
+    const Quotient q(s);
+    unsigned long long bad_code = 0, bad_bits = 0, bad_tiny = 0;
+    uint32_t first = 0, first_bits = 0;
+    for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
+        const float x = __uint_as_float(xb << 16);
+        if (!(fabsf(x) <= amax)) continue;
+        const float fast = q(x);
+        const float ref = __fdiv_rn(x, s);
+        if ((cvt_e4m3x2(fast, 0.0f) & 0xFFu) != (cvt_e4m3x2(ref, 0.0f) & 0xFFu)) {
+            if (bad_code == 0) first = (abits << 16) | xb;
+            ++bad_code;
+        }
+        if (__float_as_uint(fast) != __float_as_uint(ref)) {
+            if (fabsf(ref) >= 0x1p-12f) {
+                if (bad_bits == 0) first_bits = (abits << 16) | xb;
+                ++bad_bits;
+            } else {
+                ++bad_tiny;
+            }
+        }
+    }
+    if (bad_code && atomicAdd(&result[0], bad_code) == 0) result[1] = first;
+    if (bad_bits && atomicAdd(&result[2], bad_bits) == 0) result[3] = first_bits;
+    if (bad_tiny) atomicAdd(&result[4], bad_tiny);
 }
 
 // A wait on a barrier that nothing completes: runs into the time limit.

@@ -188,6 +188,17 @@ const char *fp8_last_cuda_error(void);
 fp8_status fp8_cast_e4m3_scaled(const float *x, float scale, uint8_t *q, int64_t n,
                                 void *stream);
 
+/* Exhaustive check of the quantizers' division path: for every positive
+ * finite bf16 amax and every bf16 x with |x| <= amax, compares the E4M3
+ * code (and the float32 quotient bits) the quantizers compute for x / s,
+ * s = amax / 448, with those of the IEEE division.  result: 5 device
+ * uint64 the caller zeroes, 16-byte aligned.  result[0] += code mismatches,
+ * result[1] = first code mismatch (amax bits << 16 | x bits), result[2] +=
+ * quotient-bit mismatches with |x / s| >= 2^-12, result[3] = first such,
+ * result[4] += quotient-bit mismatches with |x / s| < 2^-12 (a range whose
+ * codes are all zero). */
+fp8_status fp8_selftest_division(unsigned long long *result, void *stream);
+
 /* Launches one block whose only wait is on a barrier that nothing completes,
  * so that the bounded wait runs out after the current time limit and
  * records FP8_ERR_TIMEOUT in the sticky error word.  For testing the timeout

@@ -56,6 +56,17 @@ def test_cast_random_fp32_sweep():
                           f"random cast {scale}")
 
 
+def test_group_division_matches_ieee_division_exhaustively():
+    """The quantizers divide by a group's scale with one reciprocal and two
+    FMAs per element; every (bf16 amax, bf16 x) pair must give the same E4M3
+    code, and the same float32 quotient, as IEEE division."""
+    bad_code, first, bad_bits, first_bits, bad_tiny = fp8.fp8_selftest_division()
+    print(f"division self-test: code mismatches {bad_code}, quotient mismatches >= 2^-12: "
+          f"{bad_bits} (first 0x{first_bits:08x}), below 2^-12: {bad_tiny}")
+    assert bad_code == 0, f"first mismatch amax=0x{first >> 16:04x} x=0x{first & 0xffff:04x}"
+    assert bad_bits == 0, f"first quotient mismatch amax=0x{first_bits >> 16:04x} x=0x{first_bits & 0xffff:04x}"
+
+
 # ------------------------------------------------------------- quantizers
 
 @pytest.mark.parametrize("rows,cols", [(1, 128), (3, 384), (127, 256), (129, 2048), (1000, 640),
