@@ -27,6 +27,7 @@ std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_gemm_attr_done[kMaxDevices];
+std::atomic<int> g_gemm_pairs[kMaxDevices][2];   // co-resident CTA pairs per kernel
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
@@ -129,23 +130,35 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, gemm::Params p, cudaS
 
     const int flag = 1 << SCALE;
     if ((g_gemm_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
-        const cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   gemm::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             gemm::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
+        // How many CTA pairs can be resident at once: the persistent grid
+        // must not exceed it, or the last pairs would wait for a second wave.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+        cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
+        int pairs = 0;
+        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<SCALE>, &cfg);
+        if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
+        if (pairs <= 0) return cuda_fail("gemm kernel cannot be resident", cudaErrorInvalidConfiguration);
+        g_gemm_pairs[dev][SCALE].store(pairs, std::memory_order_relaxed);
         g_gemm_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
     }
+    const int max_pairs = g_gemm_pairs[dev][SCALE].load(std::memory_order_relaxed);
 
     CUtensorMap ma, mb, mc;
     if ((st = make_operand_map(&ma, a, p.M, p.K, gemm::BM)) != FP8_OK) return st;
-    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN)) != FP8_OK) return st;
+    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN / 2)) != FP8_OK) return st;
     if ((st = make_output_map(&mc, p.out, p.M, p.N)) != FP8_OK) return st;
 
-    p.tiles_m = static_cast<int>((p.M + gemm::BM - 1) / gemm::BM);
+    p.tiles_m = static_cast<int>((p.M + 2 * gemm::BM - 1) / (2 * gemm::BM));
     p.tiles_n = static_cast<int>((p.N + gemm::BN - 1) / gemm::BN);
     p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    const int grid = 2 * static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
     gemm::gemm_kernel<SCALE><<<grid, gemm::THREADS, gemm::SMEM_BYTES, stream>>>(ma, mb, mc, p);
     return last_launch_status("gemm launch");
 }

@@ -1,4 +1,4 @@
-// FP8 block-scaled GEMM on tcgen05 tensor cores (sm_100a).
+// FP8 block-scaled GEMM on tcgen05 tensor cores (sm_100a), CTA-pair version.
 //
 //   C[i, j] = sum_t  s_a(t, i) * s_b(t, j) * P_t[i, j],
 //   P_t[i, j] = sum_{k in slab t} A[i, k] * B[j, k]      (E4M3 codes)
@@ -9,25 +9,35 @@
 // leaves the tensor core in FP32 and is scaled before it joins the running
 // FP32 accumulator.
 //
-// Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
-//   warp 0      TMA producer: A tile 128 x 128 B and B tile 256 x 128 B per
-//               slab into a 4-deep ring of 128-byte-swizzled stages, plus the
-//               slab's scale vectors into an 8-deep ring (plain bulk copies;
-//               no multicast anywhere).
-//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=32, E4M3 ->
-//               F32) per slab into one of two 256-column TMEM buffers, fresh
-//               for every slab; commits free the smem stage and publish the
-//               TMEM buffer.
-//   warps 2, 3  idle (they complete warpgroup 0, which gives registers away)
-//   warps 4..11 promotion + epilogue: each thread owns one output row (TMEM
-//               lane) and 128 columns, pulls the slab partials with
-//               tcgen05.ld (two 32-column loads per wait), releases the TMEM
-//               buffer as soon as the last load has landed, and does
-//               acc = fma(s_a * s_b, P, acc) in registers with packed FP32x2
-//               FMAs.  After the last slab it rounds to BF16 into a per-warp
-//               128-byte-swizzled staging buffer that TMA stores to global
-//               memory asynchronously.  TMEM double buffering lets promotion
-//               of slab t overlap the MMAs of slab t+1.
+// Structure: clusters of two CTAs (one per SM) compute 256 x 256 output
+// tiles; persistent, 384 threads (3 warpgroups) per CTA.
+//   warp 0      operand producer (both CTAs): TMA loads of this CTA's 128
+//               rows of A and 128 rows of B per slab into a 4-deep ring of
+//               128-byte-swizzled stages, counted on the leader CTA's
+//               barrier (plain loads; no multicast anywhere).
+//   warp 2      scale producer (both CTAs): the scale vectors of 8 slabs at
+//               a time into a CTA-local 2-slot ring by bulk copy, paced by
+//               the epilogue (one wait and one arrive per 8 slabs), so a slow
+//               epilogue never holds up the operand loads.
+//   warps 1, 3  MMA issuers (leader CTA only), warp 1 for even slabs and warp
+//               3 for odd slabs: 4 x tcgen05.mma.cta_group::2 (M=256, N=256,
+//               K=32, E4M3 -> F32) per slab into the slab's 256-column TMEM
+//               buffer (two, alternating), fresh every slab; each CTA's TMEM
+//               receives its 128 rows.  Commits free both CTAs' smem stage
+//               and publish the TMEM buffer to both CTAs' epilogues.  Issuing
+//               one slab takes ~400 clocks (each MMA ~75, each commit ~60)
+//               against 512 clocks of tensor work, so two issuers keep the
+//               wait for a returned buffer off the tensor pipe's path.
+//   warps 4..11 promotion + epilogue (both CTAs): each thread owns one output
+//               row (TMEM lane) and 128 columns, pulls the slab partials with
+//               tcgen05.ld (loads one 32-column chunk ahead of the FMAs),
+//               hands the TMEM buffer back to the leader as soon as the last
+//               chunk has landed,
+//               and does acc = fma(s_a * s_b, P, acc) in registers with packed
+//               FP32x2 FMAs.  After the last slab it rounds to BF16 into a
+//               per-warp 128-byte-swizzled staging buffer that TMA stores to
+//               global memory asynchronously.  TMEM double buffering lets
+//               promotion of slab t overlap the MMAs of slab t+1.
 // Scale modes:
 //   kScaleRowBlock (fprop, dgrad): s_a is per output row (1x128 activation
 //     groups), s_b per 128-column block of the weight (128x128 blocks), so
@@ -35,8 +45,9 @@
 //   kScaleOuter (wgrad): both operands are grouped along tokens, so the
 //     coefficient is the outer product s_a(t, i) * s_b(t, j).
 // Every mbarrier wait is bounded in time (see mbar_wait); on a time-out the
-// block stops issuing work, drains the copies and MMAs it has in flight,
-// frees its tensor memory and exits.
+// CTA stops issuing work, drains the copies and MMAs it has in flight, meets
+// its partner at the closing cluster barrier, frees its tensor memory and
+// exits.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -46,15 +57,17 @@
 namespace fp8blk {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;              // output rows per CTA (256 per pair)
+constexpr int BN = 256;              // output columns per pair tile
 constexpr int BK = 128;              // one quantization slab
 constexpr int UMMA_K = 32;           // K of one kind::f8f6f4 MMA
-constexpr int STAGES = 3;
-constexpr int SSTAGES = 8;
-constexpr int A_BYTES = BM * BK;
-constexpr int B_BYTES = BN * BK;
+constexpr int STAGES = 4;
+constexpr int SCHUNK = 8;            // slabs of scales per ring slot
+constexpr int SSLOTS = 2;            // scale ring slots
+constexpr int A_BYTES = BM * BK;             // this CTA's 128 rows of A
+constexpr int B_BYTES = (BN / 2) * BK;       // this CTA's 128 rows of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_WARP0 = 4;         // first epilogue warp (warpgroups 1 and 2)
 constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
@@ -67,23 +80,23 @@ constexpr int REGS_EPILOGUE = 232;
 static_assert(128 * REGS_PRODUCER + 256 * REGS_EPILOGUE <= THREADS * REGS_LAUNCH,
               "register split exceeds the launch allocation");
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int SCALE_SLOT_BYTES = (BM + BN) * 4;
+constexpr int SCALE_SLOT_BYTES = SCHUNK * (BM + BN) * 4;   // s_a then s_b, slab-major
 constexpr int MAX_KB = 256;          // slabs of a fprop/dgrad contraction
 constexpr int SB_REGS = MAX_KB / 32;
-
 constexpr int OUT_WARP_BYTES = 32 * 128 * 2;     // 32 rows x 128 BF16 per epilogue warp
 
 constexpr int OFF_SCALES = STAGES * STAGE_BYTES;
-constexpr int OFF_OUT = OFF_SCALES + SSTAGES * SCALE_SLOT_BYTES;
+constexpr int OFF_OUT = OFF_SCALES + SSLOTS * SCALE_SLOT_BYTES;
 constexpr int OFF_BARS = OFF_OUT + EPI_WARPS * OUT_WARP_BYTES;
-constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 * SSTAGES + 1;
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 * SSLOTS + 1;
 constexpr int OFF_TMEM_SLOT = OFF_BARS + NUM_BARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(OFF_OUT % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzled stages must be 1024-byte aligned");
 
-constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
+constexpr uint32_t IDESC = idesc_e4m3_f32(2 * BM, BN);
 
 enum ScaleMode : int { kScaleRowBlock = 0, kScaleOuter = 1 };
 
@@ -95,7 +108,7 @@ struct Params {
     int64_t sb_ld;
     __nv_bfloat16* out;     // [M, N]
     int M, N, K;            // output rows, output columns, contraction
-    int tiles_m, tiles_n;
+    int tiles_m, tiles_n;   // pair tiles: 256-row by 256-column
     uint64_t wait_ns;
 };
 
@@ -141,7 +154,7 @@ __device__ __forceinline__ void load_sb(float (&regs)[SB_REGS], const Params& p,
 }
 
 template <int SCALE>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -150,6 +163,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();            // 0 = leader of the pair
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
     const int num_kb = p.K / BK;
     const int total_tiles = p.tiles_m * p.tiles_n;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
@@ -160,29 +176,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     bars.tfull = bars.empty + 8 * STAGES;
     bars.tempty = bars.tfull + 16;
     bars.sfull = bars.tempty + 16;
-    bars.sempty = bars.sfull + 8 * SSTAGES;
-    bars.drain = bars.sempty + 8 * SSTAGES;
+    bars.sempty = bars.sfull + 8 * SSLOTS;
+    bars.drain = bars.sempty + 8 * SSLOTS;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(bars.full_(s), 1);
-            mbar_init(bars.empty_(s), 1);
+            mbar_init(bars.full_(s), 1);      // leader: its producer's arrive + both CTAs' bytes
+            mbar_init(bars.empty_(s), 1);     // one multicast commit
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars.tfull_(b), 1);
-            mbar_init(bars.tempty_(b), EPI_WARPS);
+            mbar_init(bars.tempty_(b), 2 * EPI_WARPS);   // leader: both CTAs' epilogue warps
         }
-        for (int s = 0; s < SSTAGES; ++s) {
+        for (int s = 0; s < SSLOTS; ++s) {
             mbar_init(bars.sfull_(s), 1);
             mbar_init(bars.sempty_(s), EPI_WARPS);
         }
-        mbar_init(bars.drain, 1);
+        mbar_init(bars.drain, 2);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(sbase + OFF_TMEM_SLOT, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(sbase + OFF_TMEM_SLOT, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmA);
@@ -190,23 +206,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         prefetch_tensormap(&tmC);
     }
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    cluster_sync();                                      // barriers and TMEM ready in both CTAs
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
 
     if (warp < EPI_WARP0) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
       if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ---------------------------------------------------- operand producer
         if (lane == 0) {
+            const uint32_t full_leader = map_to_cta(bars.full, 0);
             int it = 0;    // slabs whose operand tiles were requested
-            int its = 0;   // slabs whose scale vectors were requested
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-                const int m0 = (tile / p.tiles_n) * BM;
+            for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+                const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
                 const int n0 = (tile % p.tiles_n) * BN;
-                const uint32_t sb_bytes =
-                    (SCALE == kScaleOuter) ? static_cast<uint32_t>(min(BN, p.N - n0)) * 4u : 0u;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     const int s = it % STAGES;
                     if (!mbar_wait(bars.empty_(s), ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
@@ -214,41 +229,70 @@ __global__ void __launch_bounds__(THREADS, 1)
                         break;
                     }
                     const uint32_t a_dst = sbase + s * STAGE_BYTES;
-                    mbar_arrive_expect_tx(bars.full_(s), STAGE_BYTES);
-                    tma_load_2d(a_dst, &tmA, kb * BK, m0, bars.full_(s));
-                    tma_load_2d(a_dst + A_BYTES, &tmB, kb * BK, n0, bars.full_(s));
+                    if (rank == 0) mbar_arrive_expect_tx(bars.full_(s), PAIR_STAGE_BYTES);
+                    tma_load_2d_pair(a_dst, &tmA, kb * BK, m_own, full_leader + 8 * s);
+                    tma_load_2d_pair(a_dst + A_BYTES, &tmB, kb * BK, n0 + static_cast<int>(rank) * (BN / 2),
+                                     full_leader + 8 * s);
                     ++it;
-
-                    const int ss = its % SSTAGES;
-                    if (!mbar_wait(bars.sempty_(ss), ((its / SSTAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t slot = sbase + OFF_SCALES + ss * SCALE_SLOT_BYTES;
-                    mbar_arrive_expect_tx(bars.sfull_(ss), BM * 4 + sb_bytes);
-                    bulk_load(slot, p.sa + static_cast<int64_t>(kb) * p.sa_ld + m0, BM * 4,
-                              bars.sfull_(ss));
-                    if (SCALE == kScaleOuter)
-                        bulk_load(slot + BM * 4, p.sb + static_cast<int64_t>(kb) * p.sb_ld + n0,
-                                  sb_bytes, bars.sfull_(ss));
-                    ++its;
                 }
             }
             if (!ok) {
-                // Let every copy already requested land before the block exits.
-                for (int j = max(0, it - STAGES); j < it; ++j)
-                    drain_wait(bars.full_(j % STAGES), (j / STAGES) & 1, p.wait_ns);
-                for (int j = max(0, its - SSTAGES); j < its; ++j)
-                    drain_wait(bars.sfull_(j % SSTAGES), (j / SSTAGES) & 1, p.wait_ns);
+                // Let every copy already requested land before the pair exits.
+                if (rank == 0) {
+                    for (int j = max(0, it - STAGES); j < it; ++j)
+                        drain_wait(bars.full_(j % STAGES), (j / STAGES) & 1, p.wait_ns);
+                } else {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 200000ull) {
+                    }
+                }
             }
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
+      } else if (warp == 2) {
+        // ------------------------------------------------------ scale producer
         if (lane == 0) {
+            int ic = 0;    // scale chunks requested
+            bool ok = true;
+            for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+                const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
+                const int n0 = (tile % p.tiles_n) * BN;
+                const uint32_t sa_bytes = (m_own < p.M) ? BM * 4u : 0u;
+                const uint32_t sb_bytes =
+                    (SCALE == kScaleOuter) ? static_cast<uint32_t>(min(BN, p.N - n0)) * 4u : 0u;
+                for (int kb0 = 0; kb0 < num_kb; kb0 += SCHUNK) {
+                    const int nslab = min(SCHUNK, num_kb - kb0);
+                    const int sl = ic % SSLOTS;
+                    if (!mbar_wait(bars.sempty_(sl), ((ic / SSLOTS) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t slot = sbase + OFF_SCALES + sl * SCALE_SLOT_BYTES;
+                    mbar_arrive_expect_tx(bars.sfull_(sl), nslab * (sa_bytes + sb_bytes));
+                    for (int j = 0; j < nslab; ++j) {
+                        const int64_t kb = kb0 + j;
+                        if (sa_bytes)
+                            bulk_load(slot + j * BM * 4, p.sa + kb * p.sa_ld + m_own, sa_bytes, bars.sfull_(sl));
+                        if (SCALE == kScaleOuter)
+                            bulk_load(slot + SCHUNK * BM * 4 + j * BN * 4, p.sb + kb * p.sb_ld + n0, sb_bytes,
+                                      bars.sfull_(sl));
+                    }
+                    ++ic;
+                }
+            }
+            if (!ok) {
+                for (int j = max(0, ic - SSLOTS); j < ic; ++j)
+                    drain_wait(bars.sfull_(j % SSLOTS), (j / SSLOTS) & 1, p.wait_ns);
+            }
+        }
+      } else if (warp == 1 || warp == 3) {
+        // -------------------------------------------------- MMA issuer (leader)
+        if (lane == 0 && rank == 0) {
+            const int sel = (warp == 1) ? 0 : 1;
             int it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+            for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    if ((it & 1) != sel) continue;
                     const int buf = it & 1;
                     if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
                         ok = false;
@@ -268,14 +312,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // +32 bytes along K inside the swizzled 128-byte row
                         const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        mma_f8(d_tmem, a_desc + adv, b_desc + adv, IDESC, k > 0 ? 1u : 0u);
+                        mma_f8_pair(d_tmem, a_desc + adv, b_desc + adv, IDESC, k > 0 ? 1u : 0u);
                     }
-                    mma_commit(bars.empty_(s));
-                    mma_commit(bars.tfull_(buf));
+                    mma_commit_pair(bars.empty_(s), 0x3);
+                    mma_commit_pair(bars.tfull_(buf), 0x3);
                 }
             }
-            // All MMAs of this thread done before the block may free TMEM.
-            mma_commit(bars.drain);
+            // All MMAs of both issuers done before the pair may free TMEM.
+            mma_commit_pair(bars.drain, 0x1);
             drain_wait(bars.drain, 0, p.wait_ns);
         }
         __syncwarp();
@@ -288,72 +332,90 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int half = ew >> 2;              // which 128 of the 256 columns
         const int row_in_tile = quarter * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t tempty_leader = map_to_cta(bars.tempty, 0);
 
         float sb_cur[SB_REGS], sb_next[SB_REGS];
-        if (SCALE == kScaleRowBlock) load_sb(sb_cur, p, blockIdx.x, half, num_kb, lane);
+        if (SCALE == kScaleRowBlock) load_sb(sb_cur, p, pair, half, num_kb, lane);
 
         float acc[128];
         int it = 0;
+        int ic = 0;        // scale chunks consumed
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-            const int m0 = (tile / p.tiles_n) * BM;
+        for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+            const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
             const int n0 = (tile % p.tiles_n) * BN;
-            if (SCALE == kScaleRowBlock) load_sb(sb_next, p, tile + gridDim.x, half, num_kb, lane);
+            if (SCALE == kScaleRowBlock) load_sb(sb_next, p, tile + npairs, half, num_kb, lane);
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 
             for (int kb = 0; kb < num_kb; ++kb, ++it) {
                 const int buf = it & 1;
-                const int ss = it % SSTAGES;
-                bool got = mbar_wait(bars.tfull_(buf), (it >> 1) & 1, abort_flag, p.wait_ns, kErrTimeout);
-                got = got && mbar_wait(bars.sfull_(ss), (it / SSTAGES) & 1, abort_flag, p.wait_ns, kErrTimeout);
+                const int sl = ic % SSLOTS;
+                const int j_in_chunk = kb % SCHUNK;
+                bool got = true;
+                if (j_in_chunk == 0)
+                    got = mbar_wait(bars.sfull_(sl), (ic / SSLOTS) & 1, abort_flag, p.wait_ns, kErrTimeout);
+                got = got && mbar_wait(bars.tfull_(buf), (it >> 1) & 1, abort_flag, p.wait_ns, kErrTimeout);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const float* slot =
-                    reinterpret_cast<const float*>(smem + OFF_SCALES + ss * SCALE_SLOT_BYTES);
-                const float sa = slot[row_in_tile];
+                    reinterpret_cast<const float*>(smem + OFF_SCALES + sl * SCALE_SLOT_BYTES);
+                const float sa = slot[j_in_chunk * BM + row_in_tile];
                 const uint32_t taddr = lane_base + buf * BN + half * 128;
                 float2 cpair = make_float2(0.0f, 0.0f);
                 if (SCALE == kScaleRowBlock) {
                     const float c = sa * pick_sb(sb_cur, kb);
                     cpair = make_float2(c, c);
                 }
-                const float* sbv = slot + BM + half * 128;
+                const float* sbv = slot + SCHUNK * BM + j_in_chunk * BN + half * 128;
+                // Promote 32 columns held in r (columns c0 .. c0+31 of this half).
+                auto promote = [&](const uint32_t (&r)[32], int c0) {
 #pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    uint32_t r[2][32];
-                    tmem_ld_32x32b_x32(taddr + g * 64, r[0]);
-                    tmem_ld_32x32b_x32(taddr + g * 64 + 32, r[1]);
-                    tmem_ld_wait();
-                    if (g == 1) {
-                        // Both halves of the buffer are in registers: hand it back.
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bars.tempty_(buf));
-                    }
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const int a = g * 64 + q * 32 + j;
-                            float2 cc = cpair;
-                            if (SCALE == kScaleOuter) {
-                                const float2 b2 = *reinterpret_cast<const float2*>(sbv + a);
-                                cc = __fmul2_rn(make_float2(sa, sa), b2);
-                            }
-                            const float2 v = __ffma2_rn(
-                                cc, make_float2(__uint_as_float(r[q][j]), __uint_as_float(r[q][j + 1])),
-                                make_float2(acc[a], acc[a + 1]));
-                            acc[a] = v.x;
-                            acc[a + 1] = v.y;
+                    for (int j = 0; j < 32; j += 2) {
+                        const int a = c0 + j;
+                        float2 cc = cpair;
+                        if (SCALE == kScaleOuter) {
+                            const float2 b2 = *reinterpret_cast<const float2*>(sbv + a);
+                            cc = __fmul2_rn(make_float2(sa, sa), b2);
                         }
+                        const float2 v = __ffma2_rn(
+                            cc, make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                            make_float2(acc[a], acc[a + 1]));
+                        acc[a] = v.x;
+                        acc[a + 1] = v.y;
                     }
-                }
+                };
+                // Loads run one chunk ahead of the FMAs; the buffer goes back
+                // to the MMA issuer as soon as the last chunk has landed.
+                uint32_t r0[32], r1[32], r2[32];
+                tmem_ld_32x32b_x32(taddr, r0);
+                tmem_ld_32x32b_x32(taddr + 32, r1);
+                tmem_ld_wait();
+                tmem_ld_32x32b_x32(taddr + 64, r2);
+                promote(r0, 0);
+                promote(r1, 32);
+                tmem_ld_wait();
+                tmem_ld_32x32b_x32(taddr + 96, r0);
+                promote(r2, 64);
+                tmem_ld_wait();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bars.sempty_(ss));
+                if (lane == 0) {
+                    if (rank == 0)
+                        mbar_arrive(bars.tempty_(buf));
+                    else
+                        mbar_arrive_remote(tempty_leader + 8 * buf);
+                }
+                promote(r0, 96);
+                if (j_in_chunk == SCHUNK - 1 || kb == num_kb - 1) {
+                    // last slab of this scale chunk: the slot may be refilled
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars.sempty_(sl));
+                    ++ic;
+                }
             }
             if (!ok) break;
 
@@ -361,7 +423,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             // 32 x 64 boxes, 128-byte rows, 16-byte chunk j of row r at
             // position j ^ (r % 8)), then TMA stores of the two boxes.
             const int col0 = n0 + half * 128;
-            if (col0 < p.N) {
+            if (col0 < p.N && m_own < p.M) {
                 uint8_t* stage_out = smem + OFF_OUT + ew * OUT_WARP_BYTES;
                 if (lane == 0) bulk_wait_group_read0();     // previous tile's store has read the buffer
                 __syncwarp();
@@ -385,8 +447,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __syncwarp();
                 if (lane == 0) {
                     const uint32_t src = smem_u32(stage_out);
-                    tma_store_2d(&tmC, src, col0, m0 + quarter * 32);
-                    tma_store_2d(&tmC, src + 4096, col0 + 64, m0 + quarter * 32);
+                    tma_store_2d(&tmC, src, col0, m_own + quarter * 32);
+                    tma_store_2d(&tmC, src + 4096, col0 + 64, m_own + quarter * 32);
                     bulk_commit_group();
                 }
             }
@@ -399,10 +461,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    cluster_sync();                                      // partner done with our smem and barriers
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
