@@ -119,6 +119,66 @@ fp8_status make_output_map(CUtensorMap* map, void* base, int64_t rows, int64_t c
     return FP8_OK;
 }
 
+// 2-D row-major map with a box of box_x (inner) by box_y elements.
+fp8_status make_map_2d(CUtensorMap* map, CUtensorMapDataType type, int elem_bytes, const void* base,
+                       int64_t rows, int64_t cols, uint32_t box_x, uint32_t box_y,
+                       CUtensorMapSwizzle swizzle, const char* what) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return FP8_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+    cuuint32_t box[2] = {box_x, box_y};
+    cuuint32_t estride[2] = {1u, 1u};
+    CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled(%s): CUresult %d", what, static_cast<int>(r));
+        return FP8_ERR_CUDA;
+    }
+    return FP8_OK;
+}
+
+std::atomic<int> g_tile_attr_done[kMaxDevices];
+
+// Persistent 128 x 128 tile quantizer (column-wise, both, or weight blocks).
+template <int MODE>
+fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* s_row,
+                             uint8_t* qT, float* s_col, cudaStream_t stream) {
+    int dev = 0, sms = 0;
+    fp8_status st = current_device(&dev);
+    if (st != FP8_OK) return st;
+    if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
+    const int flag = 1 << MODE;
+    if ((g_tile_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
+        const cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   tile::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(quantize)", e);
+        g_tile_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
+    }
+    CUtensorMap mx, mq, mqt;
+    if ((st = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, rows, cols, 64, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B, "quantize input")) != FP8_OK)
+        return st;
+    // Unused maps still need a valid encoding: point them at an output.
+    const void* qbase = q ? static_cast<const void*>(q) : static_cast<const void*>(qT);
+    const void* qtbase = qT ? static_cast<const void*>(qT) : static_cast<const void*>(q);
+    if ((st = make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qbase, q ? rows : cols, q ? cols : rows,
+                          128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "row codes")) != FP8_OK)
+        return st;
+    if ((st = make_map_2d(&mqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qtbase, qT ? cols : rows, qT ? rows : cols,
+                          128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "transposed codes")) != FP8_OK)
+        return st;
+    const int64_t tiles = (rows / 128) * (cols / 128);
+    const int64_t cap = 2 * static_cast<int64_t>(sms);
+    const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
+    quant_tile_kernel<MODE><<<grid, tile::THREADS, tile::SMEM_BYTES, stream>>>(
+        mx, mq, mqt, rows, cols, s_row, s_col, qT != nullptr ? 1 : 0,
+        g_wait_ns.load(std::memory_order_relaxed));
+    return last_launch_status("tile quantize launch");
+}
+
 // Shared launcher of the three GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
 // codes, both K-major; scales described by `p`.
 template <int SCALE>
@@ -209,15 +269,9 @@ fp8_status fp8_quantize_act_1x128(const void* x_bf16, int64_t rows, int64_t cols
             x, units, rows, groups, reinterpret_cast<uint2*>(q_row), s_row);
         return last_launch_status("row-wise quantize launch");
     }
-    const int64_t tiles = (rows / 128) * (cols / 128);
-    if (tiles > kMaxDim) return FP8_ERR_SHAPE;
     if (mode == FP8_COLWISE)
-        quant_tile_kernel<kTileColwise><<<static_cast<unsigned>(tiles), 256, 0, s>>>(
-            x, rows, cols, nullptr, nullptr, q_colT, s_col);
-    else
-        quant_tile_kernel<kTileBoth><<<static_cast<unsigned>(tiles), 256, 0, s>>>(
-            x, rows, cols, q_row, s_row, q_colT, s_col);
-    return last_launch_status("tile quantize launch");
+        return launch_tile_quant<kTileColwise>(x_bf16, rows, cols, nullptr, nullptr, q_colT, s_col, s);
+    return launch_tile_quant<kTileBoth>(x_bf16, rows, cols, q_row, s_row, q_colT, s_col, s);
 }
 
 fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k, uint8_t* wq,
@@ -227,11 +281,8 @@ fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k,
     if (!w_bf16 || !wq || !sw) return FP8_ERR_NULL;
     if (!aligned16(w_bf16) || !aligned16(wq) || !aligned16(sw) || (wqT && !aligned16(wqT)))
         return FP8_ERR_ALIGN;
-    const int64_t tiles = (n / 128) * (k / 128);
-    if (tiles > kMaxDim) return FP8_ERR_SHAPE;
-    quant_tile_kernel<kTileWeight><<<static_cast<unsigned>(tiles), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4*>(w_bf16), n, k, wq, nullptr, wqT, sw);
-    return last_launch_status("weight quantize launch");
+    return launch_tile_quant<kTileWeight>(w_bf16, n, k, wq, nullptr, wqT, sw,
+                                          static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_fprop(const uint8_t* xq, const float* sx, const uint8_t* wq,

@@ -9,11 +9,14 @@
 //   quant_rowwise_kernel : 1x128 groups along rows.  Each half-warp owns one
 //                          group per step (16 lanes x 16 bytes), reduces amax
 //                          with 4 shuffles and writes 8 code bytes per lane.
-//   quant_tile_kernel    : 128 x 128 tiles staged in shared memory, for
-//                          groups along columns (tokens) with transposed
-//                          output, for both groupings from one read, and for
-//                          128x128 weight blocks (+ transposed codes).
+//   quant_tile_kernel    : persistent, 128 x 128 tiles fed by TMA into a
+//                          double buffer, for groups along columns (tokens)
+//                          with transposed output, for both groupings from
+//                          one read, and for 128x128 weight blocks (+
+//                          transposed codes); codes leave by TMA stores.
 #pragma once
+
+#include <cuda_bf16.h>
 
 #include "ptx.cuh"
 
@@ -40,7 +43,9 @@ __device__ __forceinline__ float group_scale(float amax) { return __fdiv_rn(amax
 // FMA and RN(q0 + e r) is the correctly rounded quotient.  The remainder is
 // exact only while it stays a normal float, so divisors outside
 // [2^-100, 2^100] (groups of tiny or huge bf16 values) take the IEEE
-// division instead.  copysign keeps the sign of -0 / s.  An exhaustive GPU
+// division instead.  The remainder is formed negated, e' = s q0 - x, and
+// the result as q0 - e' r: the same values, and the signed zeros come out
+// right (for x = -0: q0 = -0, e' = +0, -e' r + q0 = -0).  An exhaustive GPU
 // check (fp8_selftest_division) compares the E4M3 codes and the quotient
 // bits of both paths for every (bf16 amax, bf16 x) pair a group can hold.
 struct Quotient {
@@ -55,8 +60,8 @@ struct Quotient {
     __device__ __forceinline__ float operator()(float x) const {
         if (!fast) return __fdiv_rn(x, s);
         const float q0 = x * r;
-        const float e = fmaf(-s, q0, x);
-        return copysignf(fmaf(e, r, q0), x);
+        const float e = fmaf(s, q0, -x);       // -(x - s q0), exact
+        return fmaf(-e, r, q0);
     }
 };
 
@@ -73,6 +78,48 @@ __device__ __forceinline__ uint2 encode8(const uint4& v, float s) {
     r.x = code2(bf16_lo(v.x), bf16_hi(v.x), q) | (code2(bf16_lo(v.y), bf16_hi(v.y), q) << 16);
     r.y = code2(bf16_lo(v.z), bf16_hi(v.z), q) | (code2(bf16_lo(v.w), bf16_hi(v.w), q) << 16);
     return r;
+}
+
+// The two bf16 of a 32-bit word (memory order: low half first) as floats.
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// max |x| over the 8 bf16 of a chunk, with packed bf16 min/max (exact).
+__device__ __forceinline__ float amax8_packed(const uint4& v) {
+    __nv_bfloat162 m = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+    m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.y)));
+    m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.z)));
+    m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.w)));
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&m);
+    return fmaxf(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
+// Quotients of two values by two group scales at once (the Quotient scheme
+// above on FP32x2 pairs); both scales must be in the fast range.
+struct QuotientPair {
+    float2 r, s2;
+    __device__ __forceinline__ QuotientPair(const Quotient& a, const Quotient& b)
+        : r(make_float2(a.r, b.r)), s2(make_float2(a.s, b.s)) {}
+    __device__ __forceinline__ QuotientPair(float s0, float r0, float s1, float r1)
+        : r(make_float2(r0, r1)), s2(make_float2(s0, s1)) {}
+    // E4M3 codes of the two bf16 of w (first in the low byte).
+    __device__ __forceinline__ uint32_t codes(uint32_t w) const {
+        const float2 x = unpack_bf16x2(w);
+        const float2 q0 = __fmul2_rn(x, r);
+        const float2 e = __ffma2_rn(s2, q0, make_float2(-x.x, -x.y));   // s q0 - x
+        const float2 q = __ffma2_rn(make_float2(-e.x, -e.y), r, q0);    // q0 - e r
+        return cvt_e4m3x2(q.x, q.y);
+    }
+};
+
+// Codes of the two bf16 of w with scales s0 (low) and s1 (high), any
+// scales (zero gives code 0; scales outside the fast range divide).
+__device__ __noinline__ uint32_t codes_pair_general(uint32_t w, const Quotient& a, const Quotient& b) {
+    const float2 x = unpack_bf16x2(w);
+    const float q0 = (a.s == 0.0f) ? 0.0f : a(x.x);
+    const float q1 = (b.s == 0.0f) ? 0.0f : b(x.y);
+    return cvt_e4m3x2(q0, q1);
 }
 
 __device__ __forceinline__ float halfwarp_max(float a) {
@@ -124,128 +171,253 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(const uint4* __restr
 
 enum TileMode : int { kTileColwise = 0, kTileBoth = 1, kTileWeight = 2 };
 
-// One 128 x 128 bf16 tile per block of 256 threads.
-//   kTileColwise : s_col[rows/128, cols], q_colT[cols, rows]
-//   kTileBoth    : the above plus q_row[rows, cols], s_row[cols/128, rows]
-//   kTileWeight  : q_row = codes [rows, cols], s_col = block scales
-//                  [rows/128, cols/128], q_colT = transposed codes or NULL
+namespace tile {
+constexpr int THREADS = 256;
+constexpr int BOX_BYTES = kGroup * 128;              // 128 rows x 64 bf16, 128-byte swizzle
+constexpr int IN_BYTES = 2 * BOX_BYTES;              // one bf16 tile = two boxes
+constexpr int OUT_BYTES = kGroup * kGroup;           // one tile of codes
+constexpr int OFF_IN0 = 0;
+constexpr int OFF_IN1 = OFF_IN0 + IN_BYTES;
+constexpr int OFF_ROW = OFF_IN1 + IN_BYTES;          // row-layout codes, 128-byte swizzle
+constexpr int OFF_COL = OFF_ROW + OUT_BYTES;         // transposed codes, 128-byte swizzle
+constexpr int OFF_RED = OFF_COL + OUT_BYTES;         // 4 x 128 floats of partial maxima
+constexpr int OFF_BARS = OFF_RED + 4 * kGroup * 4;
+constexpr int SMEM_BYTES = OFF_BARS + 2 * 8 + 16 + 1024;   // + alignment slack
+static_assert(OFF_ROW % 1024 == 0 && OFF_COL % 1024 == 0 && BOX_BYTES % 1024 == 0,
+              "swizzled tiles must be 1024-byte aligned");
+
+// Byte offset of 16-byte chunk `chunk` of row `r` in a 128-byte-swizzled
+// tile of 128-byte rows (the TMA 128B swizzle pattern).
+__device__ __forceinline__ int sw128(int r, int chunk) { return r * 128 + ((chunk ^ (r & 7)) << 4); }
+}  // namespace tile
+
+// Persistent quantizer of 128 x 128 bf16 tiles, two tile buffers per block
+// fed by TMA, outputs staged in shared memory and written by TMA stores.
+//   kTileColwise : groups along columns (tokens): s_col[rows/128, cols],
+//                  codes q_colT[cols, rows]
+//   kTileBoth    : the above plus groups along rows: q_row[rows, cols],
+//                  s_row[cols/128, rows], from the same read
+//   kTileWeight  : 128 x 128 blocks: q_row = codes [rows, cols], s_col =
+//                  block scales [rows/128, cols/128], transposed codes
+//                  through tmQT when has_qT
+// Maps (all 128-byte swizzle): tmX bf16 [rows, cols], box 64 x 128;
+//   tmQ u8 [rows, cols], box 128 x 128; tmQT u8 [cols, rows], box 128 x 128.
+// Row pass: threads t and t + 128 share row t % 128, 64 columns each.
+// Column pass: thread owns columns 2p, 2p+1 over the 32 rows of quarter qq.
 template <int MODE>
-__global__ void __launch_bounds__(256, 3) quant_tile_kernel(const uint4* __restrict__ x,
-                                                         int64_t rows, int64_t cols,
-                                                         uint8_t* __restrict__ q_row,
-                                                         float* __restrict__ s_row,
-                                                         uint8_t* __restrict__ q_colT,
-                                                         float* __restrict__ s_col) {
-    __shared__ __align__(16) uint32_t tile[kGroup][kGroup / 2];  // bf16 pairs, 32 KB
-    __shared__ float red[8][kGroup];
+__global__ void __launch_bounds__(tile::THREADS, 2)
+    quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmQT, int64_t rows, int64_t cols,
+                      float* __restrict__ s_row, float* __restrict__ s_col, int has_qT,
+                      uint64_t wait_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    float* red = reinterpret_cast<float*>(smem + tile::OFF_RED);
+    const uint32_t bar0 = sbase + tile::OFF_BARS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + tile::OFF_BARS + 16);
 
     const int t = threadIdx.x;
     const int lane = t & 31;
     const int warp = t >> 5;
     const int64_t tiles_c = cols / kGroup;
-    const int64_t tr = blockIdx.x / tiles_c;
-    const int64_t tc = blockIdx.x - tr * tiles_c;
-    const int64_t r0 = tr * kGroup;
-    const int64_t c0 = tc * kGroup;
+    const int64_t total = (rows / kGroup) * tiles_c;
+    const bool want_rows = (MODE != kTileColwise);
+    const bool want_cols = (MODE != kTileWeight) || has_qT;
 
-    // Load: thread t owns 16-byte chunk (t % 16) of rows t/16 + 16 i.
-    const int chunk = t & 15;
-    const int rbase = t >> 4;
-    uint4 v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int64_t row = r0 + rbase + 16 * i;
-        v[i] = __ldg(x + (row * cols + c0) / 8 + chunk);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<uint4*>(&tile[rbase + 16 * i][chunk * 4]) = v[i];
+    auto issue_load = [&](int64_t tl, int j) {
+        const uint32_t dst = sbase + (j ? tile::OFF_IN1 : tile::OFF_IN0);
+        const int32_t x = static_cast<int32_t>((tl % tiles_c) * kGroup);
+        const int32_t y = static_cast<int32_t>((tl / tiles_c) * kGroup);
+        mbar_arrive_expect_tx(bar0 + 8 * j, tile::IN_BYTES);
+        tma_load_2d(dst, &tmX, x, y, bar0 + 8 * j);
+        tma_load_2d(dst + tile::BOX_BYTES, &tmX, x + 64, y, bar0 + 8 * j);
+    };
 
-    // Row-group amax (16 lanes share a row).
-    float ramax[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ramax[i] = halfwarp_max(amax8(v[i]));
-
-    float block_scale = 0.0f;
-    if (MODE == kTileWeight) {
-        float a = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a = fmaxf(a, ramax[i]);
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
-        if (lane == 0) red[0][warp] = a;
+    if (t == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar0 + 8, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmX);
+        for (int j = 0; j < 2; ++j) {
+            const int64_t tl = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
+            if (tl < total) issue_load(tl, j);
+        }
     }
     __syncthreads();
-    if (MODE == kTileWeight) {
-        float a = red[0][0];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) a = fmaxf(a, red[0][w]);
-        block_scale = group_scale(a);
-    }
 
-    // Row-layout outputs.
-    if (MODE == kTileBoth || MODE == kTileWeight) {
+    const int rrow = t & 127;          // row-pass row
+    const int rbox = t >> 7;           // row-pass box (columns 64 rbox ..)
+    const int p = t & 63;              // column-pass column pair
+    const int qq = t >> 6;             // column-pass row quarter
+    const int pbox = p >> 5;           // box holding columns 2p, 2p+1
+    const int pchunk = (p & 31) >> 2;  // their 16-byte chunk in the row
+    const int pbyte = (p & 3) * 4;     // their bytes in the chunk
+
+    int i = 0;
+    for (int64_t tl = blockIdx.x; tl < total; tl += gridDim.x, ++i) {
+        const int b = i & 1;
+        const int64_t tr = tl / tiles_c, tc = tl - tr * tiles_c;
+        const int64_t r0 = tr * kGroup, c0 = tc * kGroup;
+        const uint8_t* tin = smem + (b ? tile::OFF_IN1 : tile::OFF_IN0);
+        bool ok = mbar_wait(bar0 + 8 * b, (i >> 1) & 1, abort_flag, wait_ns, kErrTimeout);
+        if (t == 0) bulk_wait_group_read0();         // previous tile's stores have read the staging
+        if (__syncthreads_or(!ok)) break;
+
+        // ---- row pass
+        const uint8_t* myrow = tin + rbox * tile::BOX_BYTES;
+        uint4 v[8];
+        float a = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int64_t row = r0 + rbase + 16 * i;
-            const float sc = (MODE == kTileWeight) ? block_scale : group_scale(ramax[i]);
-            *reinterpret_cast<uint2*>(q_row + row * cols + c0 + chunk * 8) = encode8(v[i], sc);
-            if (MODE == kTileBoth && chunk == 0) s_row[tc * rows + row] = sc;
+        for (int k = 0; k < 8; ++k) {
+            v[k] = *reinterpret_cast<const uint4*>(myrow + tile::sw128(rrow, k));
+            a = fmaxf(a, amax8_packed(v[k]));
         }
-        if (MODE == kTileWeight && t == 0) s_col[tr * tiles_c + tc] = block_scale;
-    }
-
-    if (MODE == kTileWeight && q_colT == nullptr) return;
-
-    // Column pass: thread owns column pair p (cols 2p, 2p+1) over the 32 rows
-    // of quarter qq.
-    const int p = t & 63;
-    const int qq = t >> 6;
-    uint32_t w[32];
-    float m0 = 0.0f, m1 = 0.0f;
+        float block_scale = 0.0f;
+        if (MODE == kTileWeight) {
 #pragma unroll
-    for (int rr = 0; rr < 32; ++rr) {
-        w[rr] = tile[qq * 32 + rr][p];
-        m0 = fmaxf(m0, fabsf(bf16_lo(w[rr])));
-        m1 = fmaxf(m1, fabsf(bf16_hi(w[rr])));
-    }
-    float s0 = block_scale, s1 = block_scale;
-    if (MODE != kTileWeight) {
-        __syncthreads();   // red[] reuse
-        red[qq][2 * p] = m0;
-        red[qq][2 * p + 1] = m1;
+            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            if (lane == 0) red[warp] = a;
+            __syncthreads();
+            a = red[0];
+#pragma unroll
+            for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w]);
+            block_scale = group_scale(a);
+            if (t == 0) s_col[tr * tiles_c + tc] = block_scale;
+            __syncthreads();                            // red[] read before reuse below
+        } else if (want_rows) {
+            red[rbox * kGroup + rrow] = a;
+            __syncthreads();
+            a = fmaxf(red[rrow], red[kGroup + rrow]);
+        }
+        if (want_rows) {
+            const float sc = (MODE == kTileWeight) ? block_scale : group_scale(a);
+            if (MODE != kTileWeight && rbox == 0) s_row[tc * rows + r0 + rrow] = sc;
+            uint8_t* orow = smem + tile::OFF_ROW;
+            const Quotient q(sc);
+            uint32_t out[16];
+            if (q.fast) {
+                const QuotientPair qp(q, q);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    out[2 * k] = qp.codes(v[k].x) | (qp.codes(v[k].y) << 16);
+                    out[2 * k + 1] = qp.codes(v[k].z) | (qp.codes(v[k].w) << 16);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    out[2 * k] = codes_pair_general(v[k].x, q, q) | (codes_pair_general(v[k].y, q, q) << 16);
+                    out[2 * k + 1] = codes_pair_general(v[k].z, q, q) | (codes_pair_general(v[k].w, q, q) << 16);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                *reinterpret_cast<uint4*>(orow + tile::sw128(rrow, 4 * rbox + k)) =
+                    make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+        }
+
+        // ---- column pass
+        if (want_cols) {
+            const uint8_t* colbase = tin + pbox * tile::BOX_BYTES + pbyte;
+            __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+#pragma unroll 8
+            for (int rr = 0; rr < 32; ++rr) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(colbase + tile::sw128(qq * 32 + rr, pchunk));
+                m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
+            }
+            float s0 = block_scale, s1 = block_scale, rc0, rc1;
+            if (MODE != kTileWeight) {
+                const uint32_t mu = *reinterpret_cast<const uint32_t*>(&m2);
+                __syncthreads();                        // red[] free again
+                red[qq * kGroup + 2 * p] = __uint_as_float(mu << 16);
+                red[qq * kGroup + 2 * p + 1] = __uint_as_float(mu & 0xFFFF0000u);
+                __syncthreads();
+                // one thread per column finishes its scale and reciprocal
+                float* col_s = red + 2 * kGroup;        // reuses rows 2, 3 of red
+                float sc = 0.0f, rc = 0.0f;
+                if (t < kGroup) {
+                    const float am = fmaxf(fmaxf(red[t], red[kGroup + t]),
+                                           fmaxf(red[2 * kGroup + t], red[3 * kGroup + t]));
+                    sc = group_scale(am);
+                    rc = Quotient(sc).r;
+                }
+                __syncthreads();                        // all partial maxima read
+                if (t < kGroup) {
+                    col_s[t] = sc;
+                    col_s[kGroup + t] = rc;
+                }
+                __syncthreads();
+                s0 = col_s[2 * p];
+                s1 = col_s[2 * p + 1];
+                rc0 = col_s[kGroup + 2 * p];
+                rc1 = col_s[kGroup + 2 * p + 1];
+                if (qq == 0)
+                    *reinterpret_cast<float2*>(s_col + tr * cols + c0 + 2 * p) = make_float2(s0, s1);
+            } else {
+                const Quotient qb(block_scale);
+                rc0 = rc1 = qb.r;
+            }
+            const Quotient q0(s0), q1(s1);
+            const bool fast = q0.fast && q1.fast;
+            const QuotientPair qp(s0, rc0, s1, rc1);
+            uint8_t* ocol = smem + tile::OFF_COL;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {               // 16-token chunks 2qq + h
+                uint32_t b0[4], b1[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t c[4];                      // codes (col 2p low byte, 2p+1 high byte)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int r = qq * 32 + h * 16 + 4 * j + u;
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(colbase + tile::sw128(r, pchunk));
+                        c[u] = fast ? qp.codes(w) : codes_pair_general(w, q0, q1);
+                    }
+                    // gather: bytes of column 2p (low) and 2p+1 (high), rows 4j..4j+3
+                    const uint32_t lo01 = __byte_perm(c[0], c[1], 0x0040);  // c0.b0, c1.b0
+                    const uint32_t lo23 = __byte_perm(c[2], c[3], 0x0040);
+                    const uint32_t hi01 = __byte_perm(c[0], c[1], 0x0051);  // c0.b1, c1.b1
+                    const uint32_t hi23 = __byte_perm(c[2], c[3], 0x0051);
+                    b0[j] = __byte_perm(lo01, lo23, 0x5410);
+                    b1[j] = __byte_perm(hi01, hi23, 0x5410);
+                }
+                const int chunk = 2 * qq + h;
+                const int c_a = 2 * p, c_b = 2 * p + 1;
+                *reinterpret_cast<uint4*>(ocol + tile::sw128(c_a, chunk)) = make_uint4(b0[0], b0[1], b0[2], b0[3]);
+                *reinterpret_cast<uint4*>(ocol + tile::sw128(c_b, chunk)) = make_uint4(b1[0], b1[1], b1[2], b1[3]);
+            }
+        }
+
+        // ---- stores of both code tiles, then the load two tiles ahead
+        fence_proxy_async_shared();
         __syncthreads();
-        float a0 = fmaxf(fmaxf(red[0][2 * p], red[1][2 * p]), fmaxf(red[2][2 * p], red[3][2 * p]));
-        float a1 = fmaxf(fmaxf(red[0][2 * p + 1], red[1][2 * p + 1]),
-                         fmaxf(red[2][2 * p + 1], red[3][2 * p + 1]));
-        s0 = group_scale(a0);
-        s1 = group_scale(a1);
-        if (qq == 0)
-            *reinterpret_cast<float2*>(s_col + tr * cols + c0 + 2 * p) = make_float2(s0, s1);
-    }
-
-    // Transposed codes: 32 consecutive tokens of columns 2p and 2p+1.
-    uint32_t b0[8], b1[8];
-    const Quotient q0(s0), q1(s1);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t wa = w[4 * j], wb = w[4 * j + 1], wc = w[4 * j + 2], wd = w[4 * j + 3];
-        if (s0 == 0.0f) {
-            b0[j] = 0u;
-        } else {
-            b0[j] = code2(bf16_lo(wa), bf16_lo(wb), q0) | (code2(bf16_lo(wc), bf16_lo(wd), q0) << 16);
-        }
-        if (s1 == 0.0f) {
-            b1[j] = 0u;
-        } else {
-            b1[j] = code2(bf16_hi(wa), bf16_hi(wb), q1) | (code2(bf16_hi(wc), bf16_hi(wd), q1) << 16);
+        if (t == 0) {
+            if (want_rows)
+                tma_store_2d(&tmQ, sbase + tile::OFF_ROW, static_cast<int32_t>(c0), static_cast<int32_t>(r0));
+            if (want_cols)
+                tma_store_2d(&tmQT, sbase + tile::OFF_COL, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
+            bulk_commit_group();
+            const int64_t nxt = tl + 2 * static_cast<int64_t>(gridDim.x);
+            if (nxt < total) issue_load(nxt, b);
         }
     }
-    uint8_t* dst0 = q_colT + (c0 + 2 * p) * rows + r0 + qq * 32;
-    uint8_t* dst1 = dst0 + rows;
-    reinterpret_cast<uint4*>(dst0)[0] = make_uint4(b0[0], b0[1], b0[2], b0[3]);
-    reinterpret_cast<uint4*>(dst0)[1] = make_uint4(b0[4], b0[5], b0[6], b0[7]);
-    reinterpret_cast<uint4*>(dst1)[0] = make_uint4(b1[0], b1[1], b1[2], b1[3]);
-    reinterpret_cast<uint4*>(dst1)[1] = make_uint4(b1[4], b1[5], b1[6], b1[7]);
+    if (t == 0) {
+        if (*abort_flag) {
+            // let loads already requested land before the block exits
+            for (int j = 0; j < 2; ++j) {
+                const int64_t tl = blockIdx.x + static_cast<int64_t>(i + j) * gridDim.x;
+                if (tl < total) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(bar0 + 8 * ((i + j) & 1), ((i + j) >> 1) & 1)) {
+                        if (globaltimer_ns() - t0 > wait_ns) break;
+                    }
+                }
+            }
+        }
+        bulk_wait_group0();
+    }
 }
 
 // ---------------------------------------------------------------- test support
