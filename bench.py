@@ -347,6 +347,23 @@ def run_reference(args, rank):
 
 # ----------------------------------------------------------------------- ours
 
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's device time: every rank enters this collective once."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flop_step: float, steps: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank ran `steps` steps of `flop_step` in at most `elapsed_ms`."""
+    return world * flop_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 def summarize_kernels(launches, events_by_graph, pk, peak_kind):
     """Per kind: launches, total ms, share, and roofline numbers."""
     kinds = {}
@@ -426,17 +443,13 @@ def main_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), device, world)
     err = fp8.fp8_get_error()
     if err != 0:
         raise RuntimeError(f"device error word {err} after the timed region")
 
     kinds = summarize_kernels(launches, events_by_graph[: min(ngraphs, args.steps)], pk, peak_kind)
-    value = world * flop_step * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_tflops(world, flop_step, args.steps, elapsed_ms)
 
     # ---- end-to-end through host buffers
     e2e = None
@@ -445,12 +458,8 @@ def main_ours(args, rank, world, local_rank):
             g.reset()
         graphs.clear()
         e2e = run_e2e(args, lib, sweep, device, world)
-        if world > 1:
-            t = torch.tensor([e2e.pop("_elapsed_ms")], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e["value"] = world * flop_step * args.e2e_steps / (float(t.item()) * 1e-3) / 1e12
-        else:
-            e2e.pop("_elapsed_ms")
+        e2e_ms = max_over_ranks(e2e.pop("_elapsed_ms"), device, world)
+        e2e["value"] = job_tflops(world, flop_step, args.e2e_steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
     dom_kind = max(kinds, key=lambda k: kinds[k]["ms"])
