@@ -33,8 +33,8 @@
 //               tcgen05.ld (loads one 32-column chunk ahead of the FMAs),
 //               hands the TMEM buffer back to the leader as soon as the last
 //               chunk has landed,
-//               and does acc = fma(s_a * s_b, P, acc) in registers with packed
-//               FP32x2 FMAs.  After the last slab it rounds to BF16 into a
+//               and does acc = fma(s_a * s_b, P, acc) in registers with scalar
+//               FP32 FMAs.  After the last slab it rounds to BF16 into a
 //               per-warp 128-byte-swizzled staging buffer that TMA stores to
 //               global memory asynchronously.  TMEM double buffering lets
 //               promotion of slab t overlap the MMAs of slab t+1.
@@ -372,6 +372,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
                 const float* sbv = slot + SCHUNK * BM + j_in_chunk * BN + half * 128;
                 // Promote 32 columns held in r (columns c0 .. c0+31 of this half).
+                // (Scalar FFMAs: the packed FP32x2 form costs extra moves to
+                // pair up registers and measured slower here.)
                 auto promote = [&](const uint32_t (&r)[32], int c0) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
@@ -381,11 +383,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             const float2 b2 = *reinterpret_cast<const float2*>(sbv + a);
                             cc = __fmul2_rn(make_float2(sa, sa), b2);
                         }
-                        const float2 v = __ffma2_rn(
-                            cc, make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
-                            make_float2(acc[a], acc[a + 1]));
-                        acc[a] = v.x;
-                        acc[a + 1] = v.y;
+                        acc[a] = fmaf(cc.x, __uint_as_float(r[j]), acc[a]);
+                        acc[a + 1] = fmaf(cc.y, __uint_as_float(r[j + 1]), acc[a + 1]);
                     }
                 };
                 // Loads run one chunk ahead of the FMAs; the buffer goes back
