@@ -62,9 +62,16 @@ FP8_PER_BF16 = 2.0                      # nominal dense FP8 : BF16 rate
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TOKENS = 8192
 LAYERS = 28
-# DRAM bytes per launch of each kernel from one ncu capture (dram__bytes_read.sum
-# + dram__bytes_write.sum); None until a capture of the current kernels exists.
-NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {}
+# DRAM bytes of one captured launch per kernel kind (dram__bytes_read.sum +
+# dram__bytes_write.sum from `ncu --set full`), with the launch they belong to.
+# Valid only for the kernels they were taken on; the profiles/ summaries give
+# the commands.  Remove an entry when its kernel changes.
+NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
+    "gemm_rowblock": (46.670e6 + 157.654e6,
+                      "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernels of commit 8161dc2"),
+    "quant_act": (201.435e6 + 159.898e6,
+                  "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit 8161dc2"),
+}
 
 
 def parse():
@@ -474,14 +481,18 @@ def main_ours(args, rank, world, local_rank):
         roofline = {"bound": "hbm", "kernel": dom_kind, "achieved": dom["gbs"], "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": dom["gbs"] / pk["hbm_gbs"], "peak_source": peak_kind}
     tr = NCU_TRAFFIC_BYTES_PER_LAUNCH.get(dom_kind)
-    roofline["traffic"] = tr
+    roofline["traffic"] = tr[0] if tr else None
+    if tr:
+        roofline["traffic_launch"] = tr[1]
+    roofline["achieved_over"] = f"all {dom['launches']} {dom_kind} launches of the timed steps (mixed shapes)"
     q_ms = sum(d["ms"] for k, d in kinds.items() if k.startswith("quant"))
     q_bytes = sum(d["bytes"] for k, d in kinds.items() if k.startswith("quant"))
     q_gbs = q_bytes / (q_ms * 1e-3) / 1e9 if q_ms else None
     roofline_quant = {"bound": "hbm", "kernel": "all quantizers", "achieved": q_gbs, "peak": pk["hbm_gbs"],
                       "unit": "GB/s", "frac": (q_gbs / pk["hbm_gbs"]) if q_gbs else None,
                       "peak_source": peak_kind,
-                      "traffic": None}
+                      "traffic": NCU_TRAFFIC_BYTES_PER_LAUNCH.get("quant_act", (None,))[0],
+                      "traffic_launch": NCU_TRAFFIC_BYTES_PER_LAUNCH.get("quant_act", (None, None))[1]}
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
