@@ -71,18 +71,20 @@ constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_WARP0 = 4;         // first epilogue warp (warpgroups 1 and 2)
 constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
-// Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup
-// 0 drops to 40 and the two epilogue warpgroups rise to 232:
-// 128 x 40 + 256 x 232 = 64512.
+// Register split: launched at 168 per thread (384 x 168 = 64512).  Row-block
+// mode: warpgroup 0 drops to 72 and the two epilogue warpgroups rise to 216
+// (128 x 72 + 256 x 216 = 64512); at 40 the producer roles spill.  Outer mode
+// needs more in the epilogue (the per-column scale products): 40 / 232.
 constexpr int REGS_LAUNCH = 168;
-constexpr int REGS_PRODUCER = 40;
-constexpr int REGS_EPILOGUE = 232;
-static_assert(128 * REGS_PRODUCER + 256 * REGS_EPILOGUE <= THREADS * REGS_LAUNCH,
+template <int SCALE> struct RegSplit;
+template <> struct RegSplit<0> { static constexpr int producer = 72, epilogue = 216; };
+template <> struct RegSplit<1> { static constexpr int producer = 40, epilogue = 232; };
+static_assert(128 * RegSplit<0>::producer + 256 * RegSplit<0>::epilogue <= THREADS * REGS_LAUNCH,
+              "register split exceeds the launch allocation");
+static_assert(128 * RegSplit<1>::producer + 256 * RegSplit<1>::epilogue <= THREADS * REGS_LAUNCH,
               "register split exceeds the launch allocation");
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int SCALE_SLOT_BYTES = SCHUNK * (BM + BN) * 4;   // s_a then s_b, slab-major
-constexpr int MAX_KB = 256;          // slabs of a fprop/dgrad contraction
-constexpr int SB_REGS = MAX_KB / 32;
 constexpr int OUT_WARP_BYTES = 32 * 128 * 2;     // 32 rows x 128 BF16 per epilogue warp
 
 constexpr int OFF_SCALES = STAGES * STAGE_BYTES;
@@ -127,29 +129,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (globaltimer_ns() - t0 > limit_ns) return;
-    }
-}
-
-// s_b of slab kb from the 8 per-lane registers (lane j holds slab j + 32 r).
-__device__ __forceinline__ float pick_sb(const float (&regs)[SB_REGS], int kb) {
-    float v = 0.0f;
-#pragma unroll
-    for (int r = 0; r < SB_REGS; ++r)
-        if ((kb >> 5) == r) v = regs[r];
-    return __shfl_sync(0xffffffffu, v, kb & 31);
-}
-
-__device__ __forceinline__ void load_sb(float (&regs)[SB_REGS], const Params& p, int tile,
-                                        int half, int num_kb, int lane) {
-    const int total = p.tiles_m * p.tiles_n;
-    const int nb_count = p.N / 128;
-    int nb = -1;
-    if (tile < total) nb = (tile % p.tiles_n) * (BN / 128) + half;
-#pragma unroll
-    for (int r = 0; r < SB_REGS; ++r) {
-        const int kb = lane + 32 * r;
-        regs[r] = (nb >= 0 && nb < nb_count && kb < num_kb) ? __ldg(p.sb + nb * p.sb_sn + kb * p.sb_sk)
-                                                           : 0.0f;
     }
 }
 
@@ -212,7 +191,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
 
     if (warp < EPI_WARP0) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<SCALE>::producer));
       if (warp == 0) {
         // ---------------------------------------------------- operand producer
         if (lane == 0) {
@@ -250,23 +229,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
       } else if (warp == 2) {
         // ------------------------------------------------------ scale producer
-        if (lane == 0) {
-            int ic = 0;    // scale chunks requested
-            bool ok = true;
-            for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-                const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
-                const int n0 = (tile % p.tiles_n) * BN;
-                const uint32_t sa_bytes = (m_own < p.M) ? BM * 4u : 0u;
-                const uint32_t sb_bytes =
-                    (SCALE == kScaleOuter) ? static_cast<uint32_t>(min(BN, p.N - n0)) * 4u : 0u;
-                for (int kb0 = 0; kb0 < num_kb; kb0 += SCHUNK) {
-                    const int nslab = min(SCHUNK, num_kb - kb0);
-                    const int sl = ic % SSLOTS;
-                    if (!mbar_wait(bars.sempty_(sl), ((ic / SSLOTS) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
-                        ok = false;
-                        break;
+        // Lane 0 issues the bulk copies of s_a (and, in outer mode, s_b).  In
+        // row-block mode lanes 0..15 also fetch the chunk's weight-block
+        // scales (two blocks per 256-column tile; strided in dgrad, so not a
+        // bulk copy) and store them into the slot before lane 0 arrives.
+        int ic = 0;    // scale chunks requested
+        bool ok = true;
+        for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+            const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
+            const int n0 = (tile % p.tiles_n) * BN;
+            const uint32_t sa_bytes = (m_own < p.M) ? BM * 4u : 0u;
+            const uint32_t sb_bytes =
+                (SCALE == kScaleOuter) ? static_cast<uint32_t>(min(BN, p.N - n0)) * 4u : 0u;
+            for (int kb0 = 0; kb0 < num_kb; kb0 += SCHUNK) {
+                const int nslab = min(SCHUNK, num_kb - kb0);
+                const int sl = ic % SSLOTS;
+                const bool got =
+                    mbar_wait(bars.sempty_(sl), ((ic / SSLOTS) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t slot = sbase + OFF_SCALES + sl * SCALE_SLOT_BYTES;
+                if (SCALE == kScaleRowBlock) {
+                    const int j = lane >> 1, h = lane & 1;
+                    const int nb = n0 / 128 + h;
+                    if (j < nslab) {
+                        float* dst = reinterpret_cast<float*>(smem + OFF_SCALES + sl * SCALE_SLOT_BYTES) +
+                                     SCHUNK * BM + 2 * j + h;
+                        *dst = (nb < p.N / 128) ? __ldg(p.sb + static_cast<int64_t>(nb) * p.sb_sn +
+                                                        static_cast<int64_t>(kb0 + j) * p.sb_sk)
+                                                : 0.0f;
                     }
-                    const uint32_t slot = sbase + OFF_SCALES + sl * SCALE_SLOT_BYTES;
+                    __syncwarp();
+                }
+                if (lane == 0) {
                     mbar_arrive_expect_tx(bars.sfull_(sl), nslab * (sa_bytes + sb_bytes));
                     for (int j = 0; j < nslab; ++j) {
                         const int64_t kb = kb0 + j;
@@ -276,14 +273,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             bulk_load(slot + SCHUNK * BM * 4 + j * BN * 4, p.sb + kb * p.sb_ld + n0, sb_bytes,
                                       bars.sfull_(sl));
                     }
-                    ++ic;
                 }
-            }
-            if (!ok) {
-                for (int j = max(0, ic - SSLOTS); j < ic; ++j)
-                    drain_wait(bars.sfull_(j % SSLOTS), (j / SSLOTS) & 1, p.wait_ns);
+                ++ic;
             }
         }
+        if (!ok && lane == 0) {
+            for (int j = max(0, ic - SSLOTS); j < ic; ++j)
+                drain_wait(bars.sfull_(j % SSLOTS), (j / SSLOTS) & 1, p.wait_ns);
+        }
+        __syncwarp();
       } else if (warp == 1 || warp == 3) {
         // -------------------------------------------------- MMA issuer (leader)
         if (lane == 0 && rank == 0) {
@@ -325,7 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_EPILOGUE));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<SCALE>::epilogue));
         // ----------------------------------------------- promotion + epilogue
         const int ew = warp - EPI_WARP0;
         const int quarter = warp & 3;          // TMEM lanes this warp may read
@@ -334,9 +332,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
         const uint32_t tempty_leader = map_to_cta(bars.tempty, 0);
 
-        float sb_cur[SB_REGS], sb_next[SB_REGS];
-        if (SCALE == kScaleRowBlock) load_sb(sb_cur, p, pair, half, num_kb, lane);
-
         float acc[128];
         int it = 0;
         int ic = 0;        // scale chunks consumed
@@ -344,7 +339,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
             const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
             const int n0 = (tile % p.tiles_n) * BN;
-            if (SCALE == kScaleRowBlock) load_sb(sb_next, p, tile + npairs, half, num_kb, lane);
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 
@@ -367,7 +361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const uint32_t taddr = lane_base + buf * BN + half * 128;
                 float2 cpair = make_float2(0.0f, 0.0f);
                 if (SCALE == kScaleRowBlock) {
-                    const float c = sa * pick_sb(sb_cur, kb);
+                    const float c = sa * slot[SCHUNK * BM + 2 * j_in_chunk + half];
                     cpair = make_float2(c, c);
                 }
                 const float* sbv = slot + SCHUNK * BM + j_in_chunk * BN + half * 128;
@@ -376,29 +370,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 // pair up registers and measured slower here.)
                 auto promote = [&](const uint32_t (&r)[32], int c0) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
+                    for (int j = 0; j < 32; j += 4) {
                         const int a = c0 + j;
-                        float2 cc = cpair;
+                        float2 c01 = cpair, c23 = cpair;
                         if (SCALE == kScaleOuter) {
-                            const float2 b2 = *reinterpret_cast<const float2*>(sbv + a);
-                            cc = __fmul2_rn(make_float2(sa, sa), b2);
+                            const float4 b4 = *reinterpret_cast<const float4*>(sbv + a);
+                            c01 = __fmul2_rn(make_float2(sa, sa), make_float2(b4.x, b4.y));
+                            c23 = __fmul2_rn(make_float2(sa, sa), make_float2(b4.z, b4.w));
                         }
-                        acc[a] = fmaf(cc.x, __uint_as_float(r[j]), acc[a]);
-                        acc[a + 1] = fmaf(cc.y, __uint_as_float(r[j + 1]), acc[a + 1]);
+                        acc[a + 0] = fmaf(c01.x, __uint_as_float(r[j + 0]), acc[a + 0]);
+                        acc[a + 1] = fmaf(c01.y, __uint_as_float(r[j + 1]), acc[a + 1]);
+                        acc[a + 2] = fmaf(c23.x, __uint_as_float(r[j + 2]), acc[a + 2]);
+                        acc[a + 3] = fmaf(c23.y, __uint_as_float(r[j + 3]), acc[a + 3]);
                     }
                 };
-                // Loads run one chunk ahead of the FMAs; the buffer goes back
-                // to the MMA issuer as soon as the last chunk has landed.
-                uint32_t r0[32], r1[32], r2[32];
-                tmem_ld_32x32b_x32(taddr, r0);
-                tmem_ld_32x32b_x32(taddr + 32, r1);
+                // Two 32-column register sets: chunks 0 and 1 land, chunk 2
+                // and 3 loads are issued into a set as soon as its FMAs have
+                // read it, and the buffer goes back to the MMA issuer once
+                // chunks 2 and 3 have landed (two waits per slab).
+                uint32_t ra[32], rb[32];
+                tmem_ld_32x32b_x32(taddr, ra);
+                tmem_ld_32x32b_x32(taddr + 32, rb);
                 tmem_ld_wait();
-                tmem_ld_32x32b_x32(taddr + 64, r2);
-                promote(r0, 0);
-                promote(r1, 32);
-                tmem_ld_wait();
-                tmem_ld_32x32b_x32(taddr + 96, r0);
-                promote(r2, 64);
+                promote(ra, 0);
+                tmem_ld_32x32b_x32(taddr + 64, ra);
+                promote(rb, 32);
+                tmem_ld_32x32b_x32(taddr + 96, rb);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -408,7 +405,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     else
                         mbar_arrive_remote(tempty_leader + 8 * buf);
                 }
-                promote(r0, 96);
+                promote(ra, 64);
+                promote(rb, 96);
                 if (j_in_chunk == SCHUNK - 1 || kb == num_kb - 1) {
                     // last slab of this scale chunk: the slot may be refilled
                     __syncwarp();
@@ -423,7 +421,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // position j ^ (r % 8)), then TMA stores of the two boxes.
             const int col0 = n0 + half * 128;
             if (col0 < p.N && m_own < p.M) {
-                uint8_t* stage_out = smem + OFF_OUT + ew * OUT_WARP_BYTES;
+                // The row's staging address and swizzle key come out of an
+                // opaque move, so that the compiler computes the 16 chunk
+                // addresses here instead of keeping them live across the slab loop.
+                uint32_t row_addr, key;
+                asm volatile("mov.u32 %0, %1;" : "=r"(row_addr) : "r"(smem_u32(smem + OFF_OUT + ew * OUT_WARP_BYTES) + lane * 128));
+                asm volatile("mov.u32 %0, %1;" : "=r"(key) : "r"((lane & 7) << 4));
                 if (lane == 0) bulk_wait_group_read0();     // previous tile's store has read the buffer
                 __syncwarp();
 #pragma unroll
@@ -439,21 +442,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     o.w = *reinterpret_cast<uint32_t*>(&h3);
                     const int box = j >> 6;                 // which 64-column box
                     const int chunk = (j & 63) >> 3;        // 16-byte chunk in the 128-byte row
-                    *reinterpret_cast<uint4*>(stage_out + box * 4096 + lane * 128 +
-                                              ((chunk ^ (lane & 7)) << 4)) = o;
+                    st_shared_v4(row_addr + box * 4096 + ((static_cast<uint32_t>(chunk) << 4) ^ key), o);
                 }
                 fence_proxy_async_shared();
                 __syncwarp();
                 if (lane == 0) {
-                    const uint32_t src = smem_u32(stage_out);
+                    const uint32_t src = smem_u32(smem + OFF_OUT + ew * OUT_WARP_BYTES);
                     tma_store_2d(&tmC, src, col0, m_own + quarter * 32);
                     tma_store_2d(&tmC, src + 4096, col0 + 64, m_own + quarter * 32);
                     bulk_commit_group();
                 }
-            }
-            if (SCALE == kScaleRowBlock) {
-#pragma unroll
-                for (int r = 0; r < SB_REGS; ++r) sb_cur[r] = sb_next[r];
             }
         }
         if (lane == 0) bulk_wait_group0();                 // output stores complete

@@ -301,6 +301,12 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32_at(uint32_t taddr, uint32_t (
         : "memory");
 }
 
+// 16-byte store to shared memory at a 32-bit shared-window address.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
