@@ -67,10 +67,6 @@ LAYERS = 28
 # Valid only for the kernels they were taken on; the profiles/ summaries give
 # the commands.  Remove an entry when its kernel changes.
 NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
-    "gemm_rowblock": (45.975e6 + 156.353e6,
-                      "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernels of commit 427b295"),
-    "gemm_outer": (123.173e6 + 34.727e6,
-                   "gate_up wgrad 12288x2048x8192 (algorithmic 167.8 MB); kernels of commit 427b295"),
     "quant_act": (201.435e6 + 159.898e6,
                   "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit 8161dc2"),
 }

@@ -102,6 +102,13 @@ constexpr uint32_t IDESC = idesc_e4m3_f32(2 * BM, BN);
 
 enum ScaleMode : int { kScaleRowBlock = 0, kScaleOuter = 1 };
 
+// Sleep between polls (ns) of the waits that are not on the hand-off's
+// critical path: the operand producer runs STAGES slabs ahead and the scale
+// producer a chunk of 8 slabs ahead.
+constexpr uint32_t kProducerSleepNs = 128;
+constexpr uint32_t kScaleSleepNs = 256;
+constexpr uint32_t kIssuerSleepNs = 0;
+
 struct Params {
     const float* sa;        // s_a(t, i) = sa[t * sa_ld + i]
     int64_t sa_ld;
@@ -203,7 +210,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const int n0 = (tile % p.tiles_n) * BN;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     const int s = it % STAGES;
-                    if (!mbar_wait(bars.empty_(s), ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                    if (!mbar_wait(bars.empty_(s), ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout,
+                                   kProducerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -244,8 +252,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int kb0 = 0; kb0 < num_kb; kb0 += SCHUNK) {
                 const int nslab = min(SCHUNK, num_kb - kb0);
                 const int sl = ic % SSLOTS;
-                const bool got =
-                    mbar_wait(bars.sempty_(sl), ((ic / SSLOTS) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout);
+                const bool got = mbar_wait(bars.sempty_(sl), ((ic / SSLOTS) & 1) ^ 1, abort_flag, p.wait_ns,
+                                           kErrTimeout, kScaleSleepNs);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
@@ -292,7 +300,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     if ((it & 1) != sel) continue;
                     const int buf = it & 1;
-                    if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                    if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout,
+                                   kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -378,10 +387,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             c01 = __fmul2_rn(make_float2(sa, sa), make_float2(b4.x, b4.y));
                             c23 = __fmul2_rn(make_float2(sa, sa), make_float2(b4.z, b4.w));
                         }
-                        acc[a + 0] = fmaf(c01.x, __uint_as_float(r[j + 0]), acc[a + 0]);
-                        acc[a + 1] = fmaf(c01.y, __uint_as_float(r[j + 1]), acc[a + 1]);
-                        acc[a + 2] = fmaf(c23.x, __uint_as_float(r[j + 2]), acc[a + 2]);
-                        acc[a + 3] = fmaf(c23.y, __uint_as_float(r[j + 3]), acc[a + 3]);
+                        const float2 v01 = __ffma2_rn(
+                            c01, make_float2(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1])),
+                            make_float2(acc[a + 0], acc[a + 1]));
+                        const float2 v23 = __ffma2_rn(
+                            c23, make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])),
+                            make_float2(acc[a + 2], acc[a + 3]));
+                        acc[a + 0] = v01.x;
+                        acc[a + 1] = v01.y;
+                        acc[a + 2] = v23.x;
+                        acc[a + 3] = v23.y;
                     }
                 };
                 // Two 32-column register sets: chunks 0 and 1 land, chunk 2

@@ -66,11 +66,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // time-out records error `code` and raises *abort so the block's other
 // roles stop too.  The clock is first read after 16 unsuccessful polls, so
 // short waits never pay for a timer read; the limit counts from there.
+// sleep_ns > 0 puts the thread to sleep between polls: a failed poll returns
+// within ~15 clocks, and a single thread spinning on it takes issue slots
+// from the other warps of its SM sub-partition.  Waits off the critical path
+// use it.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns, unsigned int code) {
+                                          uint64_t limit_ns, unsigned int code, uint32_t sleep_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = 0;
     for (uint32_t it = 1;; ++it) {
+        if (sleep_ns) __nanosleep(sleep_ns);
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15u) == 0) {
             if (*abort) return false;
