@@ -57,6 +57,9 @@ struct Quotient {
 #endif
         fast = (s_ >= 0x1p-100f) && (s_ <= 0x1p100f);
     }
+    // With the reciprocal RN(1/s) already at hand.
+    __device__ __forceinline__ Quotient(float s_, float r_)
+        : s(s_), r(r_), fast((s_ >= 0x1p-100f) && (s_ <= 0x1p100f)) {}
     __device__ __forceinline__ float operator()(float x) const {
         if (!fast) return __fdiv_rn(x, s);
         const float q0 = x * r;
@@ -269,12 +272,13 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
         // ---- row pass
         const uint8_t* myrow = tin + rbox * tile::BOX_BYTES;
         uint4 v[8];
-        float a = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            v[k] = *reinterpret_cast<const uint4*>(myrow + tile::sw128(rrow, k));
-            a = fmaxf(a, amax8_packed(v[k]));
-        }
+        for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const uint4*>(myrow + tile::sw128(rrow, k));
+        // pairwise tree over the 8 chunk maxima (short dependency chains)
+        float a = fmaxf(fmaxf(fmaxf(amax8_packed(v[0]), amax8_packed(v[1])),
+                              fmaxf(amax8_packed(v[2]), amax8_packed(v[3]))),
+                        fmaxf(fmaxf(amax8_packed(v[4]), amax8_packed(v[5])),
+                              fmaxf(amax8_packed(v[6]), amax8_packed(v[7]))));
         float block_scale = 0.0f;
         if (MODE == kTileWeight) {
 #pragma unroll
@@ -321,12 +325,16 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
         // ---- column pass
         if (want_cols) {
             const uint8_t* colbase = tin + pbox * tile::BOX_BYTES + pbyte;
-            __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
-#pragma unroll 8
+            // four independent running maxima, then combined
+            __nv_bfloat162 mq[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mq[u] = __float2bfloat162_rn(0.0f);
+#pragma unroll
             for (int rr = 0; rr < 32; ++rr) {
                 const uint32_t w = *reinterpret_cast<const uint32_t*>(colbase + tile::sw128(qq * 32 + rr, pchunk));
-                m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
+                mq[rr & 3] = __hmax2(mq[rr & 3], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
             }
+            const __nv_bfloat162 m2 = __hmax2(__hmax2(mq[0], mq[1]), __hmax2(mq[2], mq[3]));
             float s0 = block_scale, s1 = block_scale, rc0, rc1;
             if (MODE != kTileWeight) {
                 const uint32_t mu = *reinterpret_cast<const uint32_t*>(&m2);
@@ -359,7 +367,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
                 const Quotient qb(block_scale);
                 rc0 = rc1 = qb.r;
             }
-            const Quotient q0(s0), q1(s1);
+            const Quotient q0(s0, rc0), q1(s1, rc1);
             const bool fast = q0.fast && q1.fast;
             const QuotientPair qp(s0, rc0, s1, rc1);
             uint8_t* ocol = smem + tile::OFF_COL;
