@@ -67,8 +67,12 @@ LAYERS = 28
 # Valid only for the kernels they were taken on; the profiles/ summaries give
 # the commands.  Remove an entry when its kernel changes.
 NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
-    "quant_act": (201.435e6 + 159.898e6,
-                  "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit 8161dc2"),
+    "gemm_rowblock": (46.055e6 + 156.894e6,
+                      "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernels of commit e352e38"),
+    "gemm_outer": (123.206e6 + 34.714e6,
+                   "gate_up wgrad 12288x2048x8192 (algorithmic 167.8 MB); kernels of commit e352e38"),
+    "quant_act": (201.481e6 + 160.148e6,
+                  "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit e352e38"),
 }
 
 
