@@ -258,6 +258,13 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
     const int pbox = p >> 5;           // box holding columns 2p, 2p+1
     const int pchunk = (p & 31) >> 2;  // their 16-byte chunk in the row
     const int pbyte = (p & 3) * 4;     // their bytes in the chunk
+    // Column-pass byte offsets in a tile buffer of row qq * 32 + 8 i + u
+    // (u = 0..7) are coff[u] + 1024 i: the swizzle depends on the row only
+    // through r % 8, so eight offsets serve all 32 rows of the quarter.
+    int coff[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        coff[u] = pbox * tile::BOX_BYTES + pbyte + qq * 32 * 128 + u * 128 + ((pchunk ^ u) << 4);
 
     int i = 0;
     for (int64_t tl = blockIdx.x; tl < total; tl += gridDim.x, ++i) {
@@ -324,14 +331,13 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
 
         // ---- column pass
         if (want_cols) {
-            const uint8_t* colbase = tin + pbox * tile::BOX_BYTES + pbyte;
             // four independent running maxima, then combined
             __nv_bfloat162 mq[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) mq[u] = __float2bfloat162_rn(0.0f);
 #pragma unroll
             for (int rr = 0; rr < 32; ++rr) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(colbase + tile::sw128(qq * 32 + rr, pchunk));
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(tin + coff[rr & 7] + (rr >> 3) * 1024);
                 mq[rr & 3] = __hmax2(mq[rr & 3], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
             }
             const __nv_bfloat162 m2 = __hmax2(__hmax2(mq[0], mq[1]), __hmax2(mq[2], mq[3]));
@@ -371,19 +377,18 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
             const bool fast = q0.fast && q1.fast;
             const QuotientPair qp(s0, rc0, s1, rc1);
             uint8_t* ocol = smem + tile::OFF_COL;
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {               // 16-token chunks 2qq + h
-                uint32_t b0[4], b1[4];
+            // Codes of rows 4j .. 4j+3 of 16-token chunk 2qq + h for both
+            // columns, gathered into one word per column (row 4j lowest).
+            auto gather16 = [&](auto&& code_of, int h, uint32_t (&b0)[4], uint32_t (&b1)[4]) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     uint32_t c[4];                      // codes (col 2p low byte, 2p+1 high byte)
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int r = qq * 32 + h * 16 + 4 * j + u;
-                        const uint32_t w = *reinterpret_cast<const uint32_t*>(colbase + tile::sw128(r, pchunk));
-                        c[u] = fast ? qp.codes(w) : codes_pair_general(w, q0, q1);
+                        const int rl = h * 16 + 4 * j + u;     // row within the quarter
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(tin + coff[rl & 7] + (rl >> 3) * 1024);
+                        c[u] = code_of(w);
                     }
-                    // gather: bytes of column 2p (low) and 2p+1 (high), rows 4j..4j+3
                     const uint32_t lo01 = __byte_perm(c[0], c[1], 0x0040);  // c0.b0, c1.b0
                     const uint32_t lo23 = __byte_perm(c[2], c[3], 0x0040);
                     const uint32_t hi01 = __byte_perm(c[0], c[1], 0x0051);  // c0.b1, c1.b1
@@ -391,6 +396,14 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
                     b0[j] = __byte_perm(lo01, lo23, 0x5410);
                     b1[j] = __byte_perm(hi01, hi23, 0x5410);
                 }
+            };
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {               // 16-token chunks 2qq + h
+                uint32_t b0[4], b1[4];
+                if (fast)
+                    gather16([&](uint32_t w) { return qp.codes(w); }, h, b0, b1);
+                else
+                    gather16([&](uint32_t w) { return codes_pair_general(w, q0, q1); }, h, b0, b1);
                 const int chunk = 2 * qq + h;
                 const int c_a = 2 * p, c_b = 2 * p + 1;
                 *reinterpret_cast<uint4*>(ocol + tile::sw128(c_a, chunk)) = make_uint4(b0[0], b0[1], b0[2], b0[3]);
