@@ -184,7 +184,8 @@ constexpr int OFF_IN1 = OFF_IN0 + IN_BYTES;
 constexpr int OFF_ROW = OFF_IN1 + IN_BYTES;          // row-layout codes, 128-byte swizzle
 constexpr int OFF_COL = OFF_ROW + OUT_BYTES;         // transposed codes, 128-byte swizzle
 constexpr int OFF_RED = OFF_COL + OUT_BYTES;         // 4 x 128 floats of partial maxima
-constexpr int OFF_BARS = OFF_RED + 4 * kGroup * 4;
+constexpr int OFF_COLS = OFF_RED + 4 * kGroup * 4;   // 128 column scales, then their reciprocals
+constexpr int OFF_BARS = OFF_COLS + 2 * kGroup * 4;
 constexpr int SMEM_BYTES = OFF_BARS + 2 * 8 + 16 + 1024;   // + alignment slack
 static_assert(OFF_ROW % 1024 == 0 && OFF_COL % 1024 == 0 && BOX_BYTES % 1024 == 0,
               "swizzled tiles must be 1024-byte aligned");
@@ -251,8 +252,10 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
     }
     __syncthreads();
 
-    const int rrow = t & 127;          // row-pass row
-    const int rbox = t >> 7;           // row-pass box (columns 64 rbox ..)
+    // Row pass: lanes l and l + 16 of a warp share row (l % 16) + 16 warp,
+    // one box (64 columns) each, so their maxima combine with one shuffle.
+    const int rrow = (lane & 15) + 16 * warp;
+    const int rbox = lane >> 4;        // row-pass box (columns 64 rbox ..)
     const int p = t & 63;              // column-pass column pair
     const int qq = t >> 6;             // column-pass row quarter
     const int pbox = p >> 5;           // box holding columns 2p, 2p+1
@@ -299,9 +302,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
             if (t == 0) s_col[tr * tiles_c + tc] = block_scale;
             __syncthreads();                            // red[] read before reuse below
         } else if (want_rows) {
-            red[rbox * kGroup + rrow] = a;
-            __syncthreads();
-            a = fmaxf(red[rrow], red[kGroup + rrow]);
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
         }
         if (want_rows) {
             const float sc = (MODE == kTileWeight) ? block_scale : group_scale(a);
@@ -344,23 +345,19 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
             float s0 = block_scale, s1 = block_scale, rc0, rc1;
             if (MODE != kTileWeight) {
                 const uint32_t mu = *reinterpret_cast<const uint32_t*>(&m2);
-                __syncthreads();                        // red[] free again
+                // (red[] and col_s[] were last read before the previous
+                // tile's closing barrier)
                 red[qq * kGroup + 2 * p] = __uint_as_float(mu << 16);
                 red[qq * kGroup + 2 * p + 1] = __uint_as_float(mu & 0xFFFF0000u);
                 __syncthreads();
                 // one thread per column finishes its scale and reciprocal
-                float* col_s = red + 2 * kGroup;        // reuses rows 2, 3 of red
-                float sc = 0.0f, rc = 0.0f;
+                float* col_s = reinterpret_cast<float*>(smem + tile::OFF_COLS);
                 if (t < kGroup) {
                     const float am = fmaxf(fmaxf(red[t], red[kGroup + t]),
                                            fmaxf(red[2 * kGroup + t], red[3 * kGroup + t]));
-                    sc = group_scale(am);
-                    rc = Quotient(sc).r;
-                }
-                __syncthreads();                        // all partial maxima read
-                if (t < kGroup) {
+                    const float sc = group_scale(am);
                     col_s[t] = sc;
-                    col_s[kGroup + t] = rc;
+                    col_s[kGroup + t] = Quotient(sc).r;
                 }
                 __syncthreads();
                 s0 = col_s[2 * p];
