@@ -71,8 +71,8 @@ NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
                       "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernels of commit e352e38"),
     "gemm_outer": (123.206e6 + 34.714e6,
                    "gate_up wgrad 12288x2048x8192 (algorithmic 167.8 MB); kernels of commit e352e38"),
-    "quant_act": (201.481e6 + 160.148e6,
-                  "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit e352e38"),
+    "quant_act": (201.454e6 + 161.469e6,
+                  "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit c40872f"),
 }
 
 
