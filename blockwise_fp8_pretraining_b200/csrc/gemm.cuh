@@ -16,28 +16,30 @@
 //               128-byte-swizzled stages, counted on the leader CTA's
 //               barrier (plain loads; no multicast anywhere).
 //   warp 2      scale producer (both CTAs): the scale vectors of 8 slabs at
-//               a time into a CTA-local 2-slot ring by bulk copy, paced by
-//               the epilogue (one wait and one arrive per 8 slabs), so a slow
-//               epilogue never holds up the operand loads.
+//               a time into a CTA-local 2-slot ring by bulk copy (in row-block
+//               mode it also writes the two weight-block scales of each slab
+//               into the slot), paced by the epilogue (one wait and one
+//               arrive per 8 slabs), so a slow epilogue never holds up the
+//               operand loads.  Both producers sleep between polls.
 //   warps 1, 3  MMA issuers (leader CTA only), warp 1 for even slabs and warp
 //               3 for odd slabs: 4 x tcgen05.mma.cta_group::2 (M=256, N=256,
 //               K=32, E4M3 -> F32) per slab into the slab's 256-column TMEM
 //               buffer (two, alternating), fresh every slab; each CTA's TMEM
 //               receives its 128 rows.  Commits free both CTAs' smem stage
-//               and publish the TMEM buffer to both CTAs' epilogues.  Issuing
-//               one slab takes ~400 clocks (each MMA ~75, each commit ~60)
-//               against 512 clocks of tensor work, so two issuers keep the
-//               wait for a returned buffer off the tensor pipe's path.
+//               and publish the TMEM buffer to both CTAs' epilogues.
 //   warps 4..11 promotion + epilogue (both CTAs): each thread owns one output
-//               row (TMEM lane) and 128 columns, pulls the slab partials with
-//               tcgen05.ld (loads one 32-column chunk ahead of the FMAs),
-//               hands the TMEM buffer back to the leader as soon as the last
-//               chunk has landed,
-//               and does acc = fma(s_a * s_b, P, acc) in registers with scalar
-//               FP32 FMAs.  After the last slab it rounds to BF16 into a
-//               per-warp 128-byte-swizzled staging buffer that TMA stores to
-//               global memory asynchronously.  TMEM double buffering lets
-//               promotion of slab t overlap the MMAs of slab t+1.
+//               row (TMEM lane) and 128 columns.  Per slab it loads the
+//               partials with tcgen05.ld into two 32-column register sets
+//               (the next chunk is loaded into a set as soon as its FMAs have
+//               read it), hands the TMEM buffer back to the leader once the
+//               last chunk has landed, and does acc = fma(s_a * s_b, P, acc)
+//               in registers with packed FP32x2 FMAs.  After the last slab it
+//               rounds to BF16 into a per-warp 128-byte-swizzled staging
+//               buffer that TMA stores to global memory asynchronously.  TMEM
+//               double buffering lets promotion of slab t overlap the MMAs of
+//               slab t+1; the promotion work done while a buffer is held is
+//               what limits the kernel (two buffers give ~1024 clocks of
+//               cover for the whole hand-off).
 // Scale modes:
 //   kScaleRowBlock (fprop, dgrad): s_a is per output row (1x128 activation
 //     groups), s_b per 128-column block of the weight (128x128 blocks), so
