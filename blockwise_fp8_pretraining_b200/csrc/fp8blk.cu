@@ -19,6 +19,26 @@ static_assert(fp8blk::kErrTimeout == static_cast<unsigned int>(FP8_ERR_TIMEOUT),
 
 namespace {
 
+// Launch with programmatic stream serialization: the kernel may begin
+// launching while the preceding kernel of the stream finishes; it waits for
+// that kernel's results in griddep_wait before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+
 using namespace fp8blk;
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
@@ -173,9 +193,10 @@ fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t*
     const int64_t tiles = (rows / 128) * (cols / 128);
     const int64_t cap = 2 * static_cast<int64_t>(sms);
     const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
-    quant_tile_kernel<MODE><<<grid, tile::THREADS, tile::SMEM_BYTES, stream>>>(
-        mx, mq, mqt, rows, cols, s_row, s_col, qT != nullptr ? 1 : 0,
-        g_wait_ns.load(std::memory_order_relaxed));
+    const cudaError_t e = launch_pdl(quant_tile_kernel<MODE>, dim3(grid), dim3(tile::THREADS), tile::SMEM_BYTES,
+                                     stream, mx, mq, mqt, rows, cols, s_row, s_col, qT != nullptr ? 1 : 0,
+                                     g_wait_ns.load(std::memory_order_relaxed));
+    if (e != cudaSuccess) return cuda_fail("tile quantize launch", e);
     return last_launch_status("tile quantize launch");
 }
 
@@ -219,7 +240,9 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, gemm::Params p, cudaS
     p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int grid = 2 * static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-    gemm::gemm_kernel<SCALE><<<grid, gemm::THREADS, gemm::SMEM_BYTES, stream>>>(ma, mb, mc, p);
+    const cudaError_t e = launch_pdl(gemm::gemm_kernel<SCALE>, dim3(grid), dim3(gemm::THREADS), gemm::SMEM_BYTES,
+                                     stream, ma, mb, mc, p);
+    if (e != cudaSuccess) return cuda_fail("gemm launch", e);
     return last_launch_status("gemm launch");
 }
 
@@ -265,8 +288,10 @@ fp8_status fp8_quantize_act_1x128(const void* x_bf16, int64_t rows, int64_t cols
         int64_t blocks = (warps_needed + 7) / 8;
         const int64_t cap = static_cast<int64_t>(sms) * 8;
         if (blocks > cap) blocks = cap;
-        quant_rowwise_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-            x, units, rows, groups, reinterpret_cast<uint2*>(q_row), s_row);
+        const cudaError_t e = launch_pdl(quant_rowwise_kernel<kUnroll>, dim3(static_cast<unsigned>(blocks)),
+                                         dim3(256), 0, s, x, units, rows, groups,
+                                         reinterpret_cast<uint2*>(q_row), s_row);
+        if (e != cudaSuccess) return cuda_fail("row-wise quantize launch", e);
         return last_launch_status("row-wise quantize launch");
     }
     if (mode == FP8_COLWISE)

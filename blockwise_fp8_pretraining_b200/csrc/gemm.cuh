@@ -198,6 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     cluster_sync();                                      // barriers and TMEM ready in both CTAs
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
+    griddep_wait();                                      // inputs of the preceding kernel are complete
 
     if (warp < EPI_WARP0) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<SCALE>::producer));
@@ -474,6 +475,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) bulk_wait_group0();                 // output stores complete
     }
 
+    griddep_launch_dependents();
     tc_fence_before();
     __syncwarp();
     cluster_sync();                                      // partner done with our smem and barriers

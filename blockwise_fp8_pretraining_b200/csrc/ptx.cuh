@@ -147,6 +147,21 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ------------------------------------------------- programmatic dependent launch
+
+// Wait until the grids this one depends on (the preceding kernel of the
+// stream, when launched with programmatic stream serialization) have
+// completed and their memory is visible.  Without that launch attribute it
+// returns at once.  Every thread calls it before its first global-memory
+// access, so the prologue overlaps the preceding kernel's tail.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel of the stream begin launching (its CTAs then run their
+// prologue and wait in griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(const uint4* __restr
     const int half = lane >> 4;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    griddep_wait();                    // inputs of the preceding kernel are complete
     for (int64_t base = warp * (2 * UNROLL); base < units; base += nwarps * (2 * UNROLL)) {
         uint4 v[UNROLL];
 #pragma unroll
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
         tma_load_2d(dst + tile::BOX_BYTES, &tmX, x + 64, y, bar0 + 8 * j);
     };
 
+    griddep_wait();                    // inputs of the preceding kernel are complete
     if (t == 0) {
         mbar_init(bar0, 1);
         mbar_init(bar0 + 8, 1);
@@ -421,6 +423,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
             if (nxt < total) issue_load(nxt, b);
         }
     }
+    griddep_launch_dependents();
     if (t == 0) {
         if (*abort_flag) {
             // let loads already requested land before the block exits
