@@ -21,8 +21,11 @@ L2, so no flush is needed between steps).
 Reported (one JSON line on rank 0):
   value      GEMM TFLOP per step x steps / device time of the timed steps,
              inputs resident in HBM; each timed step replays a captured CUDA
-             graph of the step's 672 launches with event-record nodes between
-             them (per-kernel times come from those events);
+             graph of the step's 672 launches (kernels launched with
+             programmatic dependent launch, so one's prologue overlaps the
+             previous one's tail); per-kernel times come from three extra
+             replays of graphs with an event-record node between every two
+             launches, run after the timed region;
   e2e        the same metric with inputs in pinned host memory and results
              copied back: per layer, host->device copy of X, W, dY, the 24
              launches, device->host copy of Y, dX, dW, pipelined on three
