@@ -1,0 +1,76 @@
+"""Host-side arithmetic of bench.py (CPU): the work per step, the per-kernel
+breakdown and the peaks it divides by.  No GPU is involved."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_step_flops_closed_form():
+    # 28 layers x 4 linears x 3 GEMMs (fprop, dgrad, wgrad), 2 T n k each
+    T = 8192
+    per_layer = sum(3 * 2 * T * n * k for n, k in ((4096, 2048), (2048, 2048), (12288, 2048), (2048, 6144)))
+    assert bench.step_gemm_flops(28) == pytest.approx(28 * per_layer, rel=0, abs=0)
+    assert bench.step_gemm_flops(28) == pytest.approx(69.269232549888e12, rel=1e-15)
+    assert bench.step_gemm_flops(1) * 28 == bench.step_gemm_flops(28)
+
+
+class _FakeEvent:
+    def __init__(self, t_ms):
+        self.t = t_ms
+
+    def elapsed_time(self, other):
+        return other.t - self.t
+
+
+def test_kernel_breakdown_shares_and_rates():
+    launches = [
+        ("quant_act", "q", None, 0.0, 4.0e6),        # 4 MB moved
+        ("gemm_rowblock", "g", None, 2.0e12, 1.0e6),  # 2 TFLOP
+        ("quant_act", "q", None, 0.0, 4.0e6),
+        ("gemm_outer", "w", None, 1.0e12, 1.0e6),
+    ]
+    # two replays, launch durations 1, 2, 1, 4 ms in each
+    events = [[_FakeEvent(t) for t in (0.0, 1.0, 3.0, 4.0, 8.0)],
+              [_FakeEvent(t) for t in (10.0, 11.0, 13.0, 14.0, 18.0)]]
+    kinds = bench.summarize_kernels(launches, events, {}, "measured")
+    assert set(kinds) == {"quant_act", "gemm_rowblock", "gemm_outer"}
+    assert sum(d["share"] for d in kinds.values()) == pytest.approx(1.0)
+    q, g, w = kinds["quant_act"], kinds["gemm_rowblock"], kinds["gemm_outer"]
+    assert q["launches"] == 4 and g["launches"] == 2 and w["launches"] == 2
+    assert q["share"] == pytest.approx(4 / 16) and g["share"] == pytest.approx(4 / 16)
+    assert w["share"] == pytest.approx(8 / 16)
+    assert q["avg_us"] == pytest.approx(1000.0)
+    assert g["tflops"] == pytest.approx(4.0e12 / 4e-3 / 1e12)     # 1000 TFLOPS
+    assert w["tflops"] == pytest.approx(2.0e12 / 8e-3 / 1e12)     # 250 TFLOPS
+    assert q["tflops"] is None
+    assert q["gbs"] == pytest.approx(16.0e6 / 4e-3 / 1e9)         # 4 GB/s
+
+
+def test_peaks_measured_file_or_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    pk, kind = bench.peaks()
+    assert kind == "fallback" and pk == bench.FALLBACK_PEAKS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6539.5, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1376.7}))
+    pk, kind = bench.peaks()
+    assert kind == "measured" and pk["bf16_tflops_sustained"] == 1376.7
+
+
+def test_traffic_entries_name_their_launch():
+    for kind, (nbytes, what) in bench.NCU_TRAFFIC_BYTES_PER_LAUNCH.items():
+        assert kind in ("gemm_rowblock", "gemm_outer", "quant_act", "quant_weight")
+        assert nbytes > 0 and "algorithmic" in what and "commit" in what
+
+
+def test_defaults_keep_the_timing_rules(monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    args = bench.parse()
+    assert args.gpus == 1 and args.impl == "ours" and args.layers == bench.LAYERS
+    assert args.warmup >= 3 and args.steps >= 1
