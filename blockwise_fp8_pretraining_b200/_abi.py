@@ -98,6 +98,33 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream))
 
 
+def _check_devices(named, current: int, stream=None) -> None:
+    """The library launches on the current CUDA device, so every tensor (and
+    an explicit torch stream) must live there; a pointer into another GPU's
+    memory would be dereferenced by the wrong device."""
+    for name, t in named:
+        if t is not None and t.device.index != current:
+            raise ValueError(f"{name} is on {t.device} but the current CUDA device is cuda:{current}; "
+                             f"call inside torch.cuda.device({t.device.index})")
+    if isinstance(stream, torch.cuda.Stream) and stream.device.index != current:
+        raise ValueError(f"stream is on {stream.device} but the current CUDA device is cuda:{current}")
+
+
+def _launch_checks(named, stream) -> None:
+    _check_devices(named, torch.cuda.current_device(), stream)
+
+
+def _record(stream, allocated) -> None:
+    """Outputs allocated here belong to the current stream's pool; when the
+    kernel runs on another torch stream, tie their lifetime to that stream
+    too so their memory is not reused while the kernel still writes it.
+    (With a raw stream handle that is the caller's job.)"""
+    if isinstance(stream, torch.cuda.Stream):
+        for t in allocated:
+            if t is not None:
+                t.record_stream(stream)
+
+
 def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
@@ -132,6 +159,8 @@ def fp8_quantize_act_1x128(x, mode=BOTH, q_row=None, s_row=None, q_colT=None, s_
     rows, cols = x.shape
     _want(x, torch.bfloat16, (rows, cols), "x")
     dev = x.device
+    given_q_row, given_s_row = q_row is not None, s_row is not None
+    given_q_colT, given_s_col = q_colT is not None, s_col is not None
     if mode & ROWWISE:
         q_row = _out(q_row, torch.uint8, (rows, cols), dev, "q_row")
         s_row = _out(s_row, torch.float32, (cols // 128, rows), dev, "s_row")
@@ -142,6 +171,10 @@ def fp8_quantize_act_1x128(x, mode=BOTH, q_row=None, s_row=None, q_colT=None, s_
         s_col = _out(s_col, torch.float32, (rows // 128, cols), dev, "s_col")
     else:
         q_colT = s_col = None
+    _launch_checks([("x", x), ("q_row", q_row), ("s_row", s_row), ("q_colT", q_colT), ("s_col", s_col)],
+                   stream)
+    _record(stream, [t for t, given in ((q_row, given_q_row), (s_row, given_s_row),
+                                         (q_colT, given_q_colT), (s_col, given_s_col)) if not given])
     _check(lib.fp8_quantize_act_1x128(_ptr(x), rows, cols, int(mode), _ptr(q_row), _ptr(s_row),
                                       _ptr(q_colT), _ptr(s_col), _stream(stream)),
            "fp8_quantize_act_1x128")
@@ -156,10 +189,13 @@ def fp8_quantize_weight_128x128(w, wq=None, sw=None, wqT=None, transposed=True, 
         raise TypeError("w must be a 2-D bfloat16 tensor")
     n, k = w.shape
     _want(w, torch.bfloat16, (n, k), "w")
+    allocated = [t is None for t in (wq, sw, wqT)]
     wq = _out(wq, torch.uint8, (n, k), w.device, "wq")
     sw = _out(sw, torch.float32, (n // 128, k // 128), w.device, "sw")
     if wqT is not None or transposed:
         wqT = _out(wqT, torch.uint8, (k, n), w.device, "wqT")
+    _launch_checks([("w", w), ("wq", wq), ("sw", sw), ("wqT", wqT)], stream)
+    _record(stream, [t for t, a in zip((wq, sw, wqT), allocated) if a])
     _check(lib.fp8_quantize_weight_128x128(_ptr(w), n, k, _ptr(wq), _ptr(sw), _ptr(wqT),
                                            _stream(stream)),
            "fp8_quantize_weight_128x128")
@@ -176,7 +212,10 @@ def fp8_block_gemm_fprop(xq, sx, wq, sw, y=None, stream=None):
     _want(sx, torch.float32, (K // 128, M), "sx")
     _want(wq, torch.uint8, (N, K), "wq")
     _want(sw, torch.float32, (N // 128, K // 128), "sw")
+    allocated = y is None
     y = _out(y, torch.bfloat16, (M, N), xq.device, "y")
+    _launch_checks([("xq", xq), ("sx", sx), ("wq", wq), ("sw", sw), ("y", y)], stream)
+    _record(stream, [y] if allocated else [])
     _check(lib.fp8_block_gemm_fprop(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K,
                                     _stream(stream)),
            "fp8_block_gemm_fprop")
@@ -193,7 +232,10 @@ def fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=None, stream=None):
     _want(sdy, torch.float32, (N // 128, M), "sdy")
     _want(wqT, torch.uint8, (K, N), "wqT")
     _want(sw, torch.float32, (N // 128, K // 128), "sw")
+    allocated = dx is None
     dx = _out(dx, torch.bfloat16, (M, K), dyq.device, "dx")
+    _launch_checks([("dyq", dyq), ("sdy", sdy), ("wqT", wqT), ("sw", sw), ("dx", dx)], stream)
+    _record(stream, [dx] if allocated else [])
     _check(lib.fp8_block_gemm_dgrad(_ptr(dyq), _ptr(sdy), _ptr(wqT), _ptr(sw), _ptr(dx), M, N, K,
                                     _stream(stream)),
            "fp8_block_gemm_dgrad")
@@ -210,7 +252,10 @@ def fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=None, stream=None):
     _want(sdyT, torch.float32, (M // 128, N), "sdyT")
     _want(xqT, torch.uint8, (K, M), "xqT")
     _want(sxT, torch.float32, (M // 128, K), "sxT")
+    allocated = dw is None
     dw = _out(dw, torch.bfloat16, (N, K), dyqT.device, "dw")
+    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw)], stream)
+    _record(stream, [dw] if allocated else [])
     _check(lib.fp8_block_gemm_wgrad(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw), N, K, M,
                                     _stream(stream)),
            "fp8_block_gemm_wgrad")
@@ -240,12 +285,14 @@ def fp8_last_cuda_error() -> str:
         return ""
 
 
-
 def fp8_cast_e4m3_scaled(x, scale: float, q=None, stream=None):
     lib = load()
     n = x.numel()
     _want(x, torch.float32, tuple(x.shape), "x")
+    allocated = q is None
     q = _out(q, torch.uint8, tuple(x.shape), x.device, "q")
+    _launch_checks([("x", x), ("q", q)], stream)
+    _record(stream, [q] if allocated else [])
     _check(lib.fp8_cast_e4m3_scaled(_ptr(x), ctypes.c_float(scale), _ptr(q), n, _stream(stream)),
            "fp8_cast_e4m3_scaled")
     return q
