@@ -44,7 +44,7 @@ def _rank_main(rank, world, port, times, results):
 def test_max_over_ranks_and_job_throughput_gloo_world2():
     world = 2
     times = [2000.0, 2100.0]          # rank 1 is the slower replica
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:   # no fork of a process that may hold CUDA
         results = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), times, results), nprocs=world, join=True)
         got = dict(results)
