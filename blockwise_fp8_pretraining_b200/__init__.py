@@ -2,8 +2,9 @@
 
 The compute path is the CUDA library libfp8blk.so (C ABI in
 include/fp8blk.h); this package is its Python binding.  The functions carry
-the C entry points' names; see ``_abi`` for their arguments.  Nothing here falls back to a CPU or library implementation: calling
-a function without the built library raises.
+the C entry points' names; see ``_abi`` for their arguments.  Nothing here
+falls back to a CPU or library implementation: calling a function without
+the built library raises.
 """
 from ._abi import (  # noqa: F401
     BOTH,

@@ -112,3 +112,51 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(OSError):
         _abi.load()
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "fp8blk.h"
+
+#define EXPECT(call, want) do { fp8_status st_ = (call); \
+    if (st_ != (want)) { printf("FAIL %s -> %d\n", #call, (int)st_); return 1; } } while (0)
+
+int main(void) {
+    void *a16 = (void *)(uintptr_t)0x10000;      /* never dereferenced */
+    unsigned char *u = (unsigned char *)a16;
+    float *f = (float *)a16;
+    EXPECT(fp8_quantize_act_1x128(a16, 256, 2048, 0, u, f, u, f, NULL), FP8_ERR_MODE);
+    EXPECT(fp8_quantize_act_1x128(a16, 100, 256, FP8_COLWISE, NULL, NULL, u, f, NULL), FP8_ERR_SHAPE);
+    EXPECT(fp8_quantize_act_1x128(NULL, 0, 256, FP8_BOTH, NULL, NULL, NULL, NULL, NULL), FP8_OK);
+    EXPECT(fp8_quantize_weight_128x128(a16, 128, 200, u, f, NULL, NULL), FP8_ERR_SHAPE);
+    EXPECT(fp8_block_gemm_fprop(u, f, u, f, a16, 128, 128, FP8_MAX_CONTRACTION_FPROP + 128, NULL),
+           FP8_ERR_SHAPE);
+    EXPECT(fp8_block_gemm_dgrad(u, f, NULL, f, a16, 128, 128, 128, NULL), FP8_ERR_NULL);
+    EXPECT(fp8_block_gemm_wgrad(u, f, u, f, a16, 128, 128, 0, NULL), FP8_ERR_SHAPE);
+    EXPECT(fp8_set_wait_timeout_ns(0), FP8_OK);
+    if (strcmp(fp8_status_string(FP8_ERR_ALIGN), "pointer not 16-byte aligned") != 0) return 1;
+    if (fp8_last_cuda_error()[0] != '\0') return 1;
+    puts("ok");
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_gets_host_statuses(lib, tmp_path):
+    """The header is plain C99 and a C program links the library directly."""
+    import os
+    import subprocess
+
+    from blockwise_fp8_pretraining_b200 import build
+
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(build.LIB)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.dirname(build.HEADER), str(src), "-o", str(exe),
+                    "-L", libdir, "-lfp8blk", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.strip() == "ok"
