@@ -430,3 +430,53 @@ def test_row_subset_matches_full():
     dw, _ = oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT)
     dws, _ = oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=[3, 200])
     assert np.array_equal(dws, dw[[3, 200]])
+
+
+def _exact(v):
+    return Fraction(float(v))
+
+
+def test_gemm_against_exact_rational_arithmetic():
+    """fprop and wgrad of a 3-slab case against the exact value in rationals:
+    every decoded code and every float32 scale is a dyadic rational, so the
+    definition's sum can be formed with no rounding at all.  The oracle's
+    FP64 result may differ from it only by its few final roundings."""
+    x, w, _ = _quant_case(28, 128, 128, 384)
+    xq, sx = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    wq, sw = oracle.quantize_weight(syn.bf16_bits(w))
+    rows = [0, 77]
+    y, bound = oracle.gemm_fprop(xq, sx, wq, sw, rows=rows)
+    dx_, dw_ = torch_decode(xq), torch_decode(wq)
+    for ri, m in enumerate(rows):
+        for n in (0, 5, 127):
+            exact = Fraction(0)
+            exact_abs = Fraction(0)
+            for t in range(3):
+                part = sum(_exact(dx_[m, k]) * _exact(dw_[n, k]) for k in range(t * G, (t + 1) * G))
+                part_abs = sum(abs(_exact(dx_[m, k]) * _exact(dw_[n, k])) for k in range(t * G, (t + 1) * G))
+                c = _exact(sx[t, m]) * _exact(sw[n // G, t])
+                exact += c * part
+                exact_abs += abs(c) * part_abs
+            tol = 8 * 2.0 ** -53 * float(exact_abs)
+            assert abs(Fraction(y[ri, n]) - exact) <= Fraction(tol)
+            assert abs(Fraction(bound[ri, n]) - exact_abs) <= Fraction(tol)
+
+    # wgrad contracts over the 384 tokens in 3 slabs with outer-product scales
+    dyT = syn.normal_bf16((384, 128), 1e-3, syn.generator(29))
+    xT = syn.activation_bf16(384, 128, 2, 30.0, syn.generator(30))
+    dyqT, sdyT = oracle.quantize_act_colwise(syn.bf16_bits(dyT))       # [128, 384], [3, 128]
+    xqT, sxT = oracle.quantize_act_colwise(syn.bf16_bits(xT))          # [128, 384], [3, 128]
+    dw, dwb = oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=[3, 100])
+    da, db = torch_decode(dyqT), torch_decode(xqT)
+    for ri, n in enumerate((3, 100)):
+        for k in (0, 64, 127):
+            exact = Fraction(0)
+            exact_abs = Fraction(0)
+            for t in range(3):
+                for m in range(t * G, (t + 1) * G):
+                    prod = _exact(sdyT[t, n]) * _exact(da[n, m]) * _exact(sxT[t, k]) * _exact(db[k, m])
+                    exact += prod
+                    exact_abs += abs(prod)
+            tol = 8 * 2.0 ** -53 * float(exact_abs)
+            assert abs(Fraction(dw[ri, k]) - exact) <= Fraction(tol)
+            assert abs(Fraction(dwb[ri, k]) - exact_abs) <= Fraction(tol)
