@@ -12,6 +12,7 @@ on.  All bf16 inputs are passed as their uint16 bit patterns.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -26,26 +27,23 @@ _lib = None
 GROUP = 128
 
 
-def build(force: bool = False) -> str:
-    """Compile fp8_oracle.c into liboracle.so (gcc -O2, OpenMP, no fast-math)."""
-    if force or not os.path.exists(_LIB_PATH) or (
-        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile fp8_oracle.c into liboracle.so (gcc -O2, OpenMP, no fast-math).
+    `src` / `out` name another copy of the source and its library (the test
+    that plants mistakes in copies of the oracle builds them this way)."""
+    if force or not os.path.exists(out) or (
+        os.path.getmtime(out) < os.path.getmtime(src)
     ):
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        tmp = out + f".tmp{os.getpid()}"
         subprocess.check_call(
             ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-             "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+             "-fno-fast-math", "-o", tmp, src, "-lm"]
         )
-        os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+        os.replace(tmp, out)
+    return out
 
 
-def _load():
-    global _lib
-    if _lib is not None:
-        return _lib
-    build()
-    lib = ctypes.CDLL(_LIB_PATH)
+def _configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     p = ctypes.c_void_p
     i64 = ctypes.c_int64
     lib.orc_e4m3_decode.restype = ctypes.c_double
@@ -62,16 +60,34 @@ def _load():
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [p, i64, i64, p, p]
-    lib.orc_gemm_fprop.restype = ctypes.c_int
-    lib.orc_gemm_fprop.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p]
-    lib.orc_gemm_dgrad.restype = ctypes.c_int
-    lib.orc_gemm_dgrad.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p]
-    lib.orc_gemm_wgrad.restype = ctypes.c_int
-    lib.orc_gemm_wgrad.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p]
+    for name in ("orc_gemm_fprop", "orc_gemm_dgrad", "orc_gemm_wgrad"):
+        fn = getattr(lib, name)
+        fn.restype = ctypes.c_int
+        fn.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p]
     lib.orc_num_threads.restype = ctypes.c_int
     lib.orc_num_threads.argtypes = []
-    _lib = lib
     return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = _configure(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+@contextlib.contextmanager
+def library(path: str):
+    """Run every wrapper below on another build of the oracle's C source
+    (a copy with a planted mistake), then restore the real one."""
+    global _lib
+    saved = _lib
+    _lib = _configure(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
 
 
 def _ptr(a: np.ndarray):
