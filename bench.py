@@ -90,6 +90,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target length of the oracle sample")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: oracle work of all warm-up and timed steps together")
     ap.add_argument("--graphs", type=int, default=8, help="distinct captured step graphs")
     return ap.parse_args()
 
@@ -268,54 +270,80 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_sample(seconds_target: float, seed: int = 0, rows_override=None):
-    """Time the CPU oracle's GEMMs on a row sample of one layer's 12 GEMM
-    shapes (operands quantized by the oracle beforehand, not timed).
-    Returns (tflops, seconds, description, threads)."""
-    import numpy as np
-    import torch
+def calibrate_rows(run_seconds, threads: int, seconds: float, max_rows: int = TOKENS) -> int:
+    """Rows per GEMM for a sample that takes about `seconds`.
 
-    import oracle
-    from blockwise_fp8_pretraining_b200 import synthetic as syn
+    The oracle parallelises over output rows, so a sample's time only grows
+    with its rows once every thread has one: calibrate on multiples of the
+    thread count, doubling until a run takes at least half a second, and fit
+    time = a + b * rows through the last two runs.  `run_seconds(rows)`
+    times one sample.  The result is a multiple of `threads` (at least one
+    row per thread) and at most `max_rows`."""
+    threads = max(1, int(threads))
+    r = min(threads, max_rows)
+    pts = [(r, run_seconds(r))]
+    while pts[-1][1] < 0.5 and r < max_rows:
+        r = min(max_rows, 2 * r)
+        pts.append((r, run_seconds(r)))
+    r2, t2 = pts[-1]
+    slope, intercept = t2 / r2, 0.0
+    if len(pts) >= 2:
+        r1, t1 = pts[-2]
+        if t2 > t1:
+            slope = (t2 - t1) / (r2 - r1)
+            intercept = max(0.0, t2 - slope * r2)
+    rows = int((seconds - intercept) / slope) if seconds > intercept else 0
+    rows = rows // threads * threads
+    return max(min(threads, max_rows), min(max_rows, rows))
 
-    lay = syn.layer(seed)
-    prepared = []
-    for name, n, k in syn.LAYER_LINEARS:
-        t = lay[name]
-        xb, wb, dyb = syn.bf16_bits(t["x"]), syn.bf16_bits(t["w"]), syn.bf16_bits(t["dy"])
-        xq, sx = oracle.quantize_act_rowwise(xb)
-        xqT, sxT = oracle.quantize_act_colwise(xb)
-        wq, sw = oracle.quantize_weight(wb)
-        dyq, sdy = oracle.quantize_act_rowwise(dyb)
-        dyqT, sdyT = oracle.quantize_act_colwise(dyb)
-        prepared.append((name, n, k, xq, sx, xqT, sxT, wq, sw, dyq, sdy, dyqT, sdyT))
-    del lay
-    threads = oracle.num_threads()
 
-    def run(rows_per_gemm):
-        flops = 0.0
+class OracleSample:
+    """The CPU oracle's GEMMs on row samples of one layer's 12 GEMM shapes
+    (fprop, dgrad and wgrad of qkv, o_proj, gate_up and down over the
+    8192-token micro-batch).  The operands are generated and quantized by
+    the oracle once, when the object is made; that is not timed."""
+
+    def __init__(self, seed: int = 0):
+        import oracle
+        from blockwise_fp8_pretraining_b200 import synthetic as syn
+
+        self.oracle = oracle
+        lay = syn.layer(seed)
+        self.prepared = []
+        for name, n, k in syn.LAYER_LINEARS:
+            t = lay[name]
+            xb, wb, dyb = syn.bf16_bits(t["x"]), syn.bf16_bits(t["w"]), syn.bf16_bits(t["dy"])
+            xq, sx = oracle.quantize_act_rowwise(xb)
+            xqT, sxT = oracle.quantize_act_colwise(xb)
+            wq, sw = oracle.quantize_weight(wb)
+            dyq, sdy = oracle.quantize_act_rowwise(dyb)
+            dyqT, sdyT = oracle.quantize_act_colwise(dyb)
+            self.prepared.append((n, k, xq, sx, xqT, sxT, wq, sw, dyq, sdy, dyqT, sdyT))
+        self.threads = oracle.num_threads()
+
+    def run(self, rows: int):
+        """The first `rows` output rows of each GEMM; returns (flop, seconds)."""
+        import numpy as np
+
+        orc = self.oracle
+        flop = 0.0
         t0 = time.perf_counter()
-        for (name, n, k, xq, sx, xqT, sxT, wq, sw, dyq, sdy, dyqT, sdyT) in prepared:
-            r_tok = np.arange(rows_per_gemm)
-            r_n = np.arange(min(rows_per_gemm, n))
-            oracle.gemm_fprop(xq, sx, wq, sw, rows=r_tok)
-            oracle.gemm_dgrad(dyq, sdy, wq, sw, rows=r_tok)
-            oracle.gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=r_n)
-            flops += 2.0 * rows_per_gemm * n * k * 2 + 2.0 * r_n.size * k * TOKENS
-        return flops, time.perf_counter() - t0
+        for (n, k, xq, sx, xqT, sxT, wq, sw, dyq, sdy, dyqT, sdyT) in self.prepared:
+            r_tok = np.arange(rows)
+            r_n = np.arange(min(rows, n))
+            orc.gemm_fprop(xq, sx, wq, sw, rows=r_tok)
+            orc.gemm_dgrad(dyq, sdy, wq, sw, rows=r_tok)
+            orc.gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=r_n)
+            flop += 2.0 * rows * n * k * 2 + 2.0 * r_n.size * k * TOKENS
+        return flop, time.perf_counter() - t0
 
-    if rows_override is not None:
-        rows = rows_override
-    else:
-        # time per call is roughly a + b * rows (operand decoding + dot products)
-        _, t_a = run(2)
-        _, t_b = run(8)
-        slope = max((t_b - t_a) / 6.0, 1e-6)
-        rows = int(max(8, min(TOKENS, (seconds_target - (t_a - 2 * slope)) / slope)))
-    flops, secs = run(rows)
-    desc = (f"oracle fprop+dgrad+wgrad of the 4 linears of one layer, first {rows} output rows each "
-            f"(8192-token micro-batch; operands quantized by the oracle beforehand, untimed)")
-    return flops / secs / 1e12, secs, desc, threads, rows
+    def rows_for(self, seconds: float) -> int:
+        return calibrate_rows(lambda r: self.run(r)[1], self.threads, seconds)
+
+    @staticmethod
+    def describe(rows: int) -> str:
+        return (f"oracle fprop+dgrad+wgrad of the 4 linears of one layer, first {rows} output rows each "
+                f"(8192-token micro-batch; operands quantized by the oracle beforehand, untimed)")
 
 
 # ------------------------------------------------------------------ reference
@@ -323,25 +351,22 @@ def oracle_sample(seconds_target: float, seed: int = 0, rows_override=None):
 def run_reference(args, rank):
     if rank != 0:
         return 0
-    sys.path.insert(0, ROOT)
     import oracle
 
     oracle.build()
-    # size one step so that warm-up + timed steps take about two minutes
-    per_step = max(1.0, 100.0 / max(1, args.steps + args.warmup))
-    _, t_a, _, threads, _ = oracle_sample(0.0, rows_override=2)
-    _, t_b, _, _, _ = oracle_sample(0.0, rows_override=8)
-    slope = max((t_b - t_a) / 6.0, 1e-6)
-    rows = int(max(2, min(TOKENS, (per_step - (t_a - 2 * slope)) / slope)))
+    sample = OracleSample()
+    # size one step so that the warm-up and timed steps together take about
+    # args.ref_seconds of oracle work
+    rows = sample.rows_for(args.ref_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_sample(0.0, rows_override=rows)
-    total_flops = total_t = 0.0
-    desc = ""
+        sample.run(rows)
+    total_flop = total_t = 0.0
     for _ in range(args.steps):
-        tf, secs, desc, threads, _ = oracle_sample(0.0, rows_override=rows)
-        total_flops += tf * 1e12 * secs
+        flop, secs = sample.run(rows)
+        total_flop += flop
         total_t += secs
-    value = total_flops / total_t / 1e12
+    value = total_flop / total_t / 1e12
+    desc = sample.describe(rows)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
@@ -350,7 +375,8 @@ def run_reference(args, rank):
         "config": {"workload": "CPU oracle on a row sample of the Qwen3-1.7B 28-layer linear sweep's "
                                "GEMM shapes (one layer's fprop/dgrad/wgrad of qkv, o_proj, gate_up, down)",
                    "tokens": TOKENS, "rows_per_gemm": rows},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
+                         "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -521,9 +547,11 @@ def main_ours(args, rank, world, local_rank):
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        tfl, secs, desc, threads, rows = oracle_sample(args.cpu_seconds)
-        cpu = {"value": tfl, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc + f"; {secs:.1f} s"}
+        sample = OracleSample()
+        rows = sample.rows_for(args.cpu_seconds)
+        flop, secs = sample.run(rows)
+        cpu = {"value": flop / secs / 1e12, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
+               "sample": sample.describe(rows) + f"; {secs:.1f} s"}
 
     if rank == 0:
         gemm_ms = sum(d["ms"] for k, d in kinds.items() if k.startswith("gemm"))

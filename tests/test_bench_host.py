@@ -74,3 +74,60 @@ def test_defaults_keep_the_timing_rules(monkeypatch):
     args = bench.parse()
     assert args.gpus == 1 and args.impl == "ours" and args.layers == bench.LAYERS
     assert args.warmup >= 3 and args.steps >= 1
+
+
+def _wave_model(a, b, threads):
+    """Oracle-like timing: rows run in waves of `threads`, plus a fixed cost."""
+    calls = []
+
+    def run(rows):
+        calls.append(rows)
+        return a + b * -(-rows // threads)
+    return run, calls
+
+
+@pytest.mark.parametrize("threads", [1, 8, 16, 112])
+def test_calibrate_rows_hits_the_target_on_thread_multiples(threads):
+    run, calls = _wave_model(0.05, 0.02, threads)
+    rows = bench.calibrate_rows(run, threads, 10.0, max_rows=8192)
+    assert (rows % threads == 0 or rows == 8192) and threads <= rows <= 8192
+    assert all(r % threads == 0 or r == 8192 for r in calls)   # never below one row per thread
+    took = run(rows)
+    assert took <= 10.0 + 1e-9
+    assert took >= min(10.0 - 0.02, run(8192)) - 1e-9             # within one wave of the target
+
+
+def test_calibrate_rows_does_not_mistake_idle_threads_for_cheap_rows():
+    # 16 threads: 2 and 8 rows cost the same, which must not read as a zero
+    # per-row cost (that picked nearly all 8192 rows and a 90 s sample)
+    run, _ = _wave_model(0.0, 0.2, 16)
+    rows = bench.calibrate_rows(run, 16, 2.0, max_rows=8192)
+    assert rows == 160 and run(rows) == pytest.approx(2.0)
+
+
+def test_calibrate_rows_bounds():
+    run, _ = _wave_model(0.0, 1e-4, 8)
+    assert bench.calibrate_rows(run, 8, 1e6, max_rows=8192) == 8192     # all rows fit
+    run, _ = _wave_model(0.0, 5.0, 8)
+    assert bench.calibrate_rows(run, 8, 0.1, max_rows=8192) == 8        # one row per thread at least
+
+
+def test_reference_arm_prints_one_bounded_line():
+    import subprocess
+
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "2", "--warmup", "1", "--ref-seconds", "3"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 1 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    rows = d["config"]["rows_per_gemm"]
+    assert rows % d["cpu_baseline"]["cores"] == 0
+    assert d["ms_per_step"] < 5000          # about 1 s of oracle work per step was asked for
