@@ -211,14 +211,24 @@ def run_launches(lib, launches, stream_handle, events=None):
 
 # -------------------------------------------------------------------- clocks
 
+def nvidia_smi_id(local_rank: int, visible) -> str:
+    """The `nvidia-smi -i` identifier of this rank's GPU: the local rank's
+    entry of CUDA_VISIBLE_DEVICES (an index or a UUID, both of which
+    nvidia-smi accepts), else the local rank itself."""
+    if visible is None or not visible.strip():
+        return str(local_rank)
+    ids = [v.strip() for v in visible.split(",") if v.strip()]
+    return ids[local_rank] if local_rank < len(ids) else str(local_rank)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu: str):
+        self.gpu = gpu
         self.proc = None
         self.lines = []
 
@@ -474,8 +484,7 @@ def main_ours(args, rank, world, local_rank):
         graphs[w % ngraphs].replay()
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else
-                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    clocks = ClockSampler(nvidia_smi_id(local_rank, os.environ.get("CUDA_VISIBLE_DEVICES")))
     clocks.start()
     if world > 1:
         dist.barrier()

@@ -131,3 +131,24 @@ def test_reference_arm_prints_one_bounded_line():
     rows = d["config"]["rows_per_gemm"]
     assert rows % d["cpu_baseline"]["cores"] == 0
     assert d["ms_per_step"] < 5000          # about 1 s of oracle work per step was asked for
+
+
+def test_nvidia_smi_id_follows_cuda_visible_devices():
+    assert bench.nvidia_smi_id(0, None) == "0"
+    assert bench.nvidia_smi_id(3, "") == "3"
+    assert bench.nvidia_smi_id(1, "4,5") == "5"
+    assert bench.nvidia_smi_id(0, " GPU-1a2b3c4d-0000 , GPU-ffff") == "GPU-1a2b3c4d-0000"
+    assert bench.nvidia_smi_id(2, "7") == "2"
+
+
+def test_clock_sampler_summarises_reasons_and_clocks(monkeypatch):
+    cs = bench.ClockSampler("0")
+    cs.proc = type("P", (), {"terminate": lambda self: None, "wait": lambda self, timeout=None: 0})()
+    cs.lines = ["0, 1800, 1965, 900.5, 0x4, Not Active, Not Active, Not Active, Active",
+                "0, 1790, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+                "0, 1810, 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+                "garbage"]
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    got = cs.stop()
+    assert got["sm_mhz"] == 1800 and got["sm_max_mhz"] == 1965 and got["samples"] == 3
+    assert got["power_w_max"] == 990.0 and got["reasons"] == ["sw_power_cap"]
