@@ -152,3 +152,15 @@ def test_clock_sampler_summarises_reasons_and_clocks(monkeypatch):
     got = cs.stop()
     assert got["sm_mhz"] == 1800 and got["sm_max_mhz"] == 1965 and got["samples"] == 3
     assert got["power_w_max"] == 990.0 and got["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_rejects_follows_the_timing_rules():
+    ok = {"sm_mhz": 1788.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert not bench.clock_rejects(ok)
+    assert not bench.clock_rejects({"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": []})
+    for bad in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clock_rejects({"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap", bad]})
+    # stuck well below max with nothing to explain it: a leftover clock lock
+    assert bench.clock_rejects({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})
+    # no sampler: nothing to judge by
+    assert not bench.clock_rejects({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]})
