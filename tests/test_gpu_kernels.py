@@ -156,6 +156,18 @@ def test_wgrad_small(N, K, M):
     check_wgrad(dy, x, rows, output_rounding=True)
 
 
+def test_longest_contraction():
+    """The longest contraction the fprop/dgrad entry points accept (256 slabs
+    of 128), and a wgrad over as many tokens: every output element."""
+    K = fp8.MAX_CONTRACTION_FPROP
+    g = syn.generator(31)
+    check_fprop(syn.activation_bf16(256, K, K // 100, 30.0, g), syn.normal_bf16((256, K), 0.02, g))
+    # dX [128, 256] = dY [128, K] W [K, 256]: the contraction runs over K
+    check_dgrad(syn.normal_bf16((128, K), 1e-3, g), syn.normal_bf16((K, 256), 0.02, g))
+    # dW [256, 128] over K tokens
+    check_wgrad(syn.normal_bf16((K, 256), 1e-3, g), syn.activation_bf16(K, 128, 1, 30.0, g))
+
+
 def test_tiny_config_fprop_dgrad_wgrad_full():
     """X [256, 2048] (4 channels x50), W [2048, 2048], dY [256, 2048]: every
     output element of the three GEMMs against the oracle."""
