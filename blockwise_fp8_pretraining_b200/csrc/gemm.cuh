@@ -377,9 +377,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     cpair = make_float2(c, c);
                 }
                 const float* sbv = slot + SCHUNK * BM + j_in_chunk * BN + half * 128;
-                // Promote 32 columns held in r (columns c0 .. c0+31 of this half).
-                // (Scalar FFMAs: the packed FP32x2 form costs extra moves to
-                // pair up registers and measured slower here.)
+                // Promote 32 columns held in r (columns c0 .. c0+31 of this half)
+                // with packed FP32x2 FMAs: acc = c * partial + acc, two
+                // columns per instruction.
                 auto promote = [&](const uint32_t (&r)[32], int c0) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
