@@ -207,7 +207,7 @@ __device__ __forceinline__ int sw128(int r, int chunk) { return r * 128 + ((chun
 //                  through tmQT when has_qT
 // Maps (all 128-byte swizzle): tmX bf16 [rows, cols], box 64 x 128;
 //   tmQ u8 [rows, cols], box 128 x 128; tmQT u8 [cols, rows], box 128 x 128.
-// Row pass: threads t and t + 128 share row t % 128, 64 columns each.
+// Row pass: lanes l and l + 16 of warp w share row 16 w + l % 16, 64 columns each.
 // Column pass: thread owns columns 2p, 2p+1 over the 32 rows of quarter qq.
 template <int MODE>
 __global__ void __launch_bounds__(tile::THREADS, 2)
