@@ -5,7 +5,8 @@ leg may import this module.  The product path never does: it shares no code
 with the CUDA library and the library does not depend on it.
 
 The arithmetic lives in ``fp8_oracle.c`` (plain C loops, FP64 accumulation,
-OpenMP over output rows); this module builds that file with gcc when the
+OpenMP over output rows; also the SwiGLU product a fused quantize-on-output
+producer has to reproduce); this module builds that file with gcc when the
 shared object is missing and wraps it with numpy.  See the C file's header
 for the definition it follows and the passages of the Puro-2B pages it rests
 on.  All bf16 inputs are passed as their uint16 bit patterns.
@@ -66,6 +67,12 @@ def _configure(lib: ctypes.CDLL) -> ctypes.CDLL:
         fn.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p]
     lib.orc_num_threads.restype = ctypes.c_int
     lib.orc_num_threads.argtypes = []
+    lib.orc_bf16_from_double.restype = ctypes.c_uint16
+    lib.orc_bf16_from_double.argtypes = [ctypes.c_double]
+    lib.orc_silu_bf16.restype = ctypes.c_uint16
+    lib.orc_silu_bf16.argtypes = [ctypes.c_uint16]
+    lib.orc_swiglu_bf16.restype = ctypes.c_int
+    lib.orc_swiglu_bf16.argtypes = [p, i64, i64, p]
     return lib
 
 
@@ -236,3 +243,30 @@ def gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=None):
                                   None if r is None else _ptr(r), nr, _ptr(y), _ptr(b)),
            "gemm_wgrad")
     return y, b
+
+
+# ----------------------------------------------------------------- SwiGLU
+
+def bf16_from_double(v: float) -> int:
+    """Bit pattern of the bfloat16 nearest to v (ties to even)."""
+    return int(_load().orc_bf16_from_double(float(v)))
+
+
+def silu_bf16(g_bits) -> np.ndarray:
+    """silu of bfloat16 values (uint16 bit patterns), evaluated in double and
+    rounded once to bfloat16."""
+    g = np.ascontiguousarray(g_bits, dtype=np.uint16)
+    fn = _load().orc_silu_bf16
+    return np.array([fn(int(b)) for b in g.ravel()], dtype=np.uint16).reshape(g.shape)
+
+
+def swiglu_bf16(gate_up_bits: np.ndarray) -> np.ndarray:
+    """H = bf16(bf16(silu(gate)) * up) for a gate_up activation
+    [rows, 2 * ffn] (gate first).  Returns uint16 bits [rows, ffn]."""
+    x = _c(gate_up_bits, np.uint16)
+    rows, cols = x.shape
+    if cols % 2:
+        raise ValueError("gate_up must have an even number of columns")
+    h = np.empty((rows, cols // 2), np.uint16)
+    _check(_load().orc_swiglu_bf16(_ptr(x), rows, cols // 2, _ptr(h)), "swiglu_bf16")
+    return h

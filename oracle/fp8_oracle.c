@@ -411,3 +411,101 @@ int orc_num_threads(void)
     return 1;
 #endif
 }
+
+/* --------------------------------------------------------------- SwiGLU
+ *
+ * The feed-forward block of the Qwen3-1.7B configuration (named in the
+ * friendli.ai model card's model property table) is a gated SiLU unit:
+ * H = silu(gate) * up, with gate and up the two halves of the fused
+ * gate_up projection.  With activations kept in BF16 (model card,
+ * training-setup paragraph), the unfused path rounds twice:
+ * h = bf16(bf16(silu(g)) * u).  This oracle takes exactly that, with each
+ * rounding to nearest even and silu evaluated in double precision before
+ * its single rounding to bfloat16.  It is the definition a fused
+ * quantize-on-output kernel has to reproduce before its 1x128 groups are
+ * quantized as above.
+ */
+
+/* Nearest bfloat16 of the finite value hi + lo, where lo is either zero or
+ * too small to move hi across a bfloat16 rounding boundary and matters only
+ * when hi lies exactly on one (a midpoint between two bfloat16 values): then
+ * its sign says on which side the value lies.  Otherwise ties go to the even
+ * significand.  8 significant bits, float32's exponent range including its
+ * subnormals; beyond the largest finite bfloat16 the result is infinity.
+ * Returns the bit pattern. */
+static uint16_t bf16_round_split(double hi, double lo)
+{
+    uint16_t sgn = signbit(hi) ? 0x8000 : 0x0000;
+    double mag = fabs(hi);
+    int ex;
+    if (mag == 0.0)
+        return sgn;
+    (void)frexp(mag, &ex);                 /* mag in [2^(ex-1), 2^ex) */
+    int lead = ex - 1 < -126 ? -126 : ex - 1;
+    double step = ldexp(1.0, lead - 7);    /* bfloat16 spacing at mag */
+    double units = mag / step;             /* exact: a power-of-two divisor */
+    double below = floor(units);
+    double frac = units - below;
+    int up;
+    if (frac != 0.5)
+        up = frac > 0.5;
+    else if (lo != 0.0)
+        up = (lo > 0.0) == (hi > 0.0);     /* the value lies beyond the midpoint */
+    else
+        up = fmod(below, 2.0) == 1.0;      /* a true tie: to the even one */
+    double rounded = (below + (up ? 1.0 : 0.0)) * step;
+    if (rounded >= ldexp(1.0, 128))
+        return sgn | 0x7F80;
+    float as_float = (float)rounded;       /* exact: at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &as_float, sizeof u);
+    return sgn | (uint16_t)((u >> 16) & 0x7FFF);
+}
+
+/* Nearest bfloat16 of a finite double, ties to even. */
+uint16_t orc_bf16_from_double(double v)
+{
+    return bf16_round_split(v, 0.0);
+}
+
+/* silu(g) = g / (1 + e^-g) for a bfloat16 g, rounded once to bfloat16.
+ * For |g| < 2^-30 the series g/2 + g^2/4 + O(g^4) is used instead: in
+ * double, 1 + e^-g rounds to 2 - g or to 2 and the quotient loses the g^2/4
+ * term, which is what decides the rounding when g/2 is a bfloat16 midpoint
+ * (g an odd multiple of the smallest subnormal).  There g/2 is exact and the
+ * higher terms cannot reach a rounding boundary.  Elsewhere the double
+ * quotient is within a few units in its last place of silu(g), far from any
+ * bfloat16 boundary for every bfloat16 g. */
+uint16_t orc_silu_bf16(uint16_t g_bits)
+{
+    double g = (double)orc_bf16_to_float(g_bits);
+    if (fabs(g) < 0x1p-30)
+        return bf16_round_split(g / 2.0, g * g / 4.0);
+    return orc_bf16_from_double(g / (1.0 + exp(-g)));
+}
+
+/* H [rows, ffn] from a gate_up activation [rows, 2 * ffn] whose columns
+ * [0, ffn) are the gate and [ffn, 2 * ffn) the up projection.  The product
+ * of two bfloat16 values is exact in double, so h has one rounding after
+ * silu's. */
+int orc_swiglu_bf16(const uint16_t *gate_up, int64_t rows, int64_t ffn,
+                    uint16_t *h)
+{
+    if (rows < 0 || ffn < 0)
+        return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *gate = gate_up + r * 2 * ffn;
+        const uint16_t *up = gate + ffn;
+        for (int64_t j = 0; j < ffn; ++j) {
+            float gf = orc_bf16_to_float(gate[j]);
+            float uf = orc_bf16_to_float(up[j]);
+            if (!isfinite(gf) || !isfinite(uf))
+                bad = 1;
+            double s = (double)orc_bf16_to_float(orc_silu_bf16(gate[j]));
+            h[r * ffn + j] = orc_bf16_from_double(s * (double)uf);
+        }
+    }
+    return bad ? -2 : 0;
+}

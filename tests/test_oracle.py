@@ -480,3 +480,114 @@ def test_gemm_against_exact_rational_arithmetic():
             tol = 8 * 2.0 ** -53 * float(exact_abs)
             assert abs(Fraction(dw[ri, k]) - exact) <= Fraction(tol)
             assert abs(Fraction(dwb[ri, k]) - exact_abs) <= Fraction(tol)
+
+
+# -------------------------------------------------------------------- SwiGLU
+
+def _bf16_rne_exact(v: Fraction, negative: bool) -> int:
+    """Bit pattern of the bfloat16 nearest to the exact rational |v| with the
+    given sign (ties to even), by rational arithmetic alone."""
+    sign = 0x8000 if negative else 0
+    mag = abs(v)
+    if mag == 0:
+        return sign
+    e = mag.numerator.bit_length() - mag.denominator.bit_length()
+    if Fraction(2) ** e > mag:
+        e -= 1                                   # now 2^e <= mag < 2^(e+1)
+    e = max(e, -126)
+    step = Fraction(2) ** (e - 7)
+    units = mag / step
+    below = units.numerator // units.denominator
+    rest = units - below
+    pick = below + 1 if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and below % 2) else below
+    value = pick * step
+    if value >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    # encode: value = pick * 2^(e-7), pick <= 256
+    if e == -126 and pick < 128:
+        return sign | int(pick)                  # subnormal: mantissa = pick
+    if pick == 256:
+        pick, e = 128, e + 1
+    return sign | ((e + 127) << 7) | (int(pick) - 128)
+
+
+def test_bf16_from_double_matches_rational_rounding_and_torch():
+    rng = np.random.default_rng(40)
+    # float32 values (torch's float32 -> bfloat16 cast is RNE): normal,
+    # subnormal, exact midpoints and their neighbours
+    mids = (np.arange(1, 2000, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    vals = np.concatenate([rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-40, 38, 20000),
+                           mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1)),
+                           np.float32([0.0, -0.0, 1e-45, -1e-45, 3.3e38, -3.3e38])]).astype(np.float32)
+    vals = vals[np.isfinite(vals)]
+    want = syn.bf16_bits(torch.from_numpy(vals).to(torch.bfloat16))
+    got = np.array([oracle.bf16_from_double(float(v)) for v in vals], dtype=np.uint16)
+    assert np.array_equal(got, want)
+    # doubles that float32 cannot hold: rounding via float32 first would land
+    # on a bfloat16 midpoint and go the wrong way
+    for v, want_bits in [(1 + 2.0 ** -8 + 2.0 ** -30, 0x3F81), (1 + 2.0 ** -8 - 2.0 ** -30, 0x3F80),
+                         (-(1 + 3 * 2.0 ** -8 - 2.0 ** -31), 0xBF81), (2.0 ** -133 * 0.5000001, 0x0001)]:
+        assert oracle.bf16_from_double(v) == want_bits == _bf16_rne_exact(Fraction(v), v < 0)
+
+
+def _silu_bits_reference(g: float, negative: bool) -> int:
+    """bfloat16 of silu(g) from decimal arithmetic: the value is taken with
+    a relative error far below 10^-(prec-5), and the result is accepted only
+    when both ends of that interval round alike; otherwise the precision is
+    raised (at |g| ~ 1e-40, g/2 can be a bfloat16 midpoint and the deciding
+    term g^2/4 sits 40 digits further down)."""
+    import decimal
+
+    for prec in (40, 200):
+        ctx = decimal.Context(prec=prec, Emax=decimal.MAX_EMAX, Emin=decimal.MIN_EMIN, traps=[])
+        gd = decimal.Decimal(g)
+        s = ctx.divide(gd, ctx.add(decimal.Decimal(1), ctx.exp(ctx.minus(gd))))
+        if s.is_zero():
+            return 0x8000 if negative else 0
+        exact = Fraction(s)
+        eps = Fraction(1, 10 ** (prec - 5))
+        lo = _bf16_rne_exact(exact * (1 - eps), negative)
+        hi = _bf16_rne_exact(exact * (1 + eps), negative)
+        if lo == hi:
+            return lo
+    raise AssertionError(f"silu({g!r}) not decided at 200 digits")
+
+
+def test_silu_every_bf16_input_against_exact_rounding():
+    """All 65,024 finite bfloat16 g against silu(g) = g / (1 + e^-g) from
+    decimal arithmetic, rounded to bfloat16 by rational arithmetic.  For
+    |g| >= 200 the value is settled without exp: g > 0 gives
+    g (1 - e^-g / (1 + e^-g)), below g by a relative 1e-87, so the bfloat16
+    g itself; g < 0 gives a magnitude below 200 e^-200 < 1e-84, under half
+    the smallest bfloat16 subnormal, so -0."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]
+    got = oracle.silu_bf16(bits)
+    g_vals = oracle.bf16_to_float(bits).astype(np.float64)
+    for b, g, out in zip(bits, g_vals, got):
+        negative = bool(b & 0x8000)
+        if abs(g) >= 200:
+            want = int(b) if g > 0 else 0x8000
+        else:
+            want = _silu_bits_reference(float(g), negative)
+        assert int(out) == want, (hex(int(b)), float(g), hex(int(out)), hex(want))
+
+
+def test_swiglu_layout_and_product_rounding():
+    g = syn.generator(41)
+    rows, ffn = 5, 200
+    gate_up = syn.normal_bf16((rows, 2 * ffn), 1.0, g)
+    bits = syn.bf16_bits(gate_up)
+    h = oracle.swiglu_bf16(bits)
+    assert h.shape == (rows, ffn)
+    s = torch.from_numpy(oracle.silu_bf16(bits[:, :ffn]).astype(np.int16)).view(torch.bfloat16)
+    up = gate_up[:, ffn:]
+    # the product of two bfloat16 values is exact in float32; one RNE cast
+    want = syn.bf16_bits((s.float() * up.float()).to(torch.bfloat16))
+    assert np.array_equal(h, want)
+    # up = 1 gives silu itself; large gates pass up through
+    ones = np.full((1, 4), 0x3F80, np.uint16)
+    gates = to_bf16_bits(np.float32([[1.0, -1.0, 100.0, -100.0]]))
+    assert np.array_equal(oracle.swiglu_bf16(np.concatenate([gates, ones], axis=1)),
+                          oracle.silu_bf16(gates))
+    assert list(oracle.silu_bf16(gates)[0]) == [0x3F3B, 0xBE8A, 0x42C8, 0x8000]

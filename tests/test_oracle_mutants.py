@@ -73,6 +73,22 @@ MUTANTS = [
      "sw + (k / GROUP) * (N / GROUP),\n                         1,", None),
     ("wgrad: both outer-product scales from dY",
      "sdyT + n, N, sxT + k, K,", "sdyT + n, N, sdyT + n, N,", None),
+    ("bf16 rounding: ties away from zero",
+     "up = fmod(below, 2.0) == 1.0;", "up = 1;", None),
+    ("bf16 rounding: the side of a midpoint ignored",
+     "up = (lo > 0.0) == (hi > 0.0);", "up = fmod(below, 2.0) == 1.0;", None),
+    ("bf16 rounding: no subnormal spacing",
+     "int lead = ex - 1 < -126 ? -126 : ex - 1;", "int lead = ex - 1;", None),
+    ("silu: the double quotient for every g (no small-g series)",
+     "if (fabs(g) < 0x1p-30)\n        return bf16_round_split(g / 2.0, g * g / 4.0);\n", "", None),
+    ("silu: e^g instead of e^-g",
+     "return orc_bf16_from_double(g / (1.0 + exp(-g)));", "return orc_bf16_from_double(g / (1.0 + exp(g)));", None),
+    ("swiglu: gate and up swapped",
+     "double s = (double)orc_bf16_to_float(orc_silu_bf16(gate[j]));\n            h[r * ffn + j] = orc_bf16_from_double(s * (double)uf);",
+     "double s = (double)orc_bf16_to_float(orc_silu_bf16(up[j]));\n            h[r * ffn + j] = orc_bf16_from_double(s * (double)gf);", None),
+    ("swiglu: silu not rounded to bfloat16 before the product",
+     "double s = (double)orc_bf16_to_float(orc_silu_bf16(gate[j]));",
+     "double s = (double)gf / (1.0 + exp(-(double)gf));", None),
 ]
 
 
