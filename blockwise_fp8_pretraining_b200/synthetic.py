@@ -153,7 +153,10 @@ def layer(seed: int, device="cpu", tokens: int = TOKENS, gen: torch.Generator | 
 
 def swiglu_bf16(gate_up: torch.Tensor) -> torch.Tensor:
     """H = silu(gate) * up in bf16 torch ops, gate = first half of the
-    columns of a gate_up output, up = second half."""
+    columns of a gate_up output, up = second half.  This prepares the
+    down-projection input that both sides receive; torch's float32 silu is
+    not correctly rounded to bf16 on every input, so it is not the definition
+    a fused producer of H is held to."""
     half = gate_up.shape[1] // 2
     gate = gate_up[:, :half]
     up = gate_up[:, half:]
