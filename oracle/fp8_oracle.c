@@ -44,9 +44,10 @@
  *   weight w          bf16 bits [n, k]
  *   weight codes      u8  [n, k]             scales f32 [n/128, k/128]
  *
- * Every function returns 0 on success and a negative number on a bad
- * argument or a non-finite input (non-finite inputs are outside the
- * definition).
+ * Every function that fills arrays returns 0 on success and a negative
+ * number on a bad argument or a non-finite input (non-finite inputs are
+ * outside the definition); the scalar codec and rounding functions return
+ * their result.
  */
 #include <math.h>
 #include <stdint.h>
