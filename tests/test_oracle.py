@@ -591,3 +591,37 @@ def test_swiglu_layout_and_product_rounding():
     assert np.array_equal(oracle.swiglu_bf16(np.concatenate([gates, ones], axis=1)),
                           oracle.silu_bf16(gates))
     assert list(oracle.silu_bf16(gates)[0]) == [0x3F3B, 0xBE8A, 0x42C8, 0x8000]
+
+
+def test_silu_rounding_margin_allows_fp64_evaluation():
+    """For every bfloat16 g with 2^-30 <= |g| < 200, silu(g) lies at least
+    2e-9 (relative) away from every bfloat16 rounding boundary.  So any
+    evaluation with a smaller relative error, such as the double-precision
+    quotient the oracle takes there (error of a few 1e-16), rounds exactly
+    as the exact value does.  The other ranges are settled without that
+    quotient: the g/2 + g^2/4 series below 2^-30, closed forms from 200 up."""
+    import decimal
+
+    ctx = decimal.Context(prec=60, Emax=decimal.MAX_EMAX, Emin=decimal.MIN_EMIN, traps=[])
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]
+    g_vals = oracle.bf16_to_float(bits).astype(np.float64)
+    smallest, count = 1.0, 0
+    for g in g_vals:
+        if not (2.0 ** -30 <= abs(g) < 200):
+            continue
+        gd = decimal.Decimal(float(g))
+        s = Fraction(ctx.divide(gd, ctx.add(decimal.Decimal(1), ctx.exp(ctx.minus(gd)))))
+        mag = abs(s)
+        e = mag.numerator.bit_length() - mag.denominator.bit_length()
+        if Fraction(2) ** e > mag:
+            e -= 1
+        step = Fraction(2) ** (max(e, -126) - 7)
+        units = mag / step
+        below = units.numerator // units.denominator
+        # the rounding boundaries around mag: the midpoints below and above it
+        d = min(abs(mag - (below + Fraction(1, 2)) * step), abs(mag - (below - Fraction(1, 2)) * step))
+        smallest = min(smallest, float(d / mag))
+        count += 1
+    assert count > 9000
+    assert smallest > 2e-9, smallest
