@@ -93,6 +93,7 @@ def parse():
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: oracle work of all warm-up and timed steps together")
     ap.add_argument("--graphs", type=int, default=8, help="distinct captured step graphs")
+    ap.add_argument("--no-ceiling", action="store_true", help="skip the FP8 library ceiling measurement")
     return ap.parse_args()
 
 
@@ -291,6 +292,68 @@ class ClockSampler:
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(power) if power else None,
                 "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------- FP8 library ceiling
+
+CEILING_SHAPES = (("8192x8192x8192", 8192, 8192, 8192),
+                  ("gate_up_fprop_8192x12288x2048", 8192, 12288, 2048))
+
+
+def fp8_library_ceiling(device, reps: int = 20, warmup: int = 5):
+    """TFLOPS of the library's E4M3 GEMM with one scale per tensor
+    (torch._scaled_mm, a cuBLASLt kernel; no blockwise scales, no promotion)
+    at 8192^3 and at the gate_up fprop shape, timed with CUDA events on the
+    current stream, outside the timed region.  It is the measured ceiling
+    beside which the blockwise kernels' TFLOPS are read, not a path of this
+    library."""
+    import torch
+
+    out = {"kind": "torch._scaled_mm per-tensor E4M3 -> BF16 (cuBLASLt)", "reps": reps}
+    clocks = ClockSampler(nvidia_smi_id(torch.cuda.current_device(), os.environ.get("CUDA_VISIBLE_DEVICES")))
+    clocks.start()
+    try:
+        for label, m, n, k in CEILING_SHAPES:
+            g = torch.Generator(device=device)
+            g.manual_seed(7)
+            a = torch.randn((m, k), device=device, generator=g).to(torch.float8_e4m3fn)
+            b = torch.randn((n, k), device=device, generator=g).to(torch.float8_e4m3fn)
+            one = torch.ones((), device=device, dtype=torch.float32)
+
+            def run():
+                return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+            for _ in range(warmup):
+                run()
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(reps):
+                run()
+            t1.record()
+            torch.cuda.synchronize()
+            ms = t0.elapsed_time(t1) / reps
+            out[label] = {"tflops": 2.0 * m * n * k / (ms * 1e-3) / 1e12, "us": 1e3 * ms}
+            del a, b
+    except Exception as e:  # noqa: BLE001 - reported, not fatal
+        out["error"] = f"{type(e).__name__}: {e}"[:300]
+    out["clocks"] = clocks.stop()
+    return out
+
+
+def roofline_fracs(tflops: float, pk: dict, peak_kind: str, ceiling: dict | None) -> dict:
+    """A GEMM's TFLOPS as a fraction of each denominator it is read against:
+    the spec dense FP8 peak, twice the measured BF16 peaks (burst and
+    sustained; the nominal FP8:BF16 ratio) and the measured FP8 library
+    ceiling at 8192^3 and at the gate_up shape."""
+    fr = {"spec_fp8_dense_4500": tflops / FP8_DENSE_SPEC_TFLOPS,
+          f"2x_{peak_kind}_bf16_burst": tflops / (FP8_PER_BF16 * pk["bf16_tflops"]),
+          f"2x_{peak_kind}_bf16_sustained": tflops / (FP8_PER_BF16 * pk["bf16_tflops_sustained"])}
+    for label, _, _, _ in CEILING_SHAPES:
+        v = (ceiling or {}).get(label)
+        if v and v.get("tflops"):
+            fr[f"fp8_library_{label}"] = tflops / v["tflops"]
+    return fr
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -549,6 +612,9 @@ def main_ours(args, rank, world, local_rank):
         e2e_ms = max_over_ranks(e2e.pop("_elapsed_ms"), device, world)
         e2e["value"] = job_tflops(world, flop_step, args.e2e_steps, e2e_ms)
 
+    # ---- measured FP8 library ceiling (outside every timed region)
+    ceiling = None if args.no_ceiling else fp8_library_ceiling(device)
+
     # ---- roofline of the dominant kernel
     dom_kind = max(kinds, key=lambda k: kinds[k]["ms"])
     dom = kinds[dom_kind]
@@ -557,7 +623,8 @@ def main_ours(args, rank, world, local_rank):
         roofline = {"bound": "tensor", "kernel": dom_kind, "achieved": dom["tflops"], "peak": fp8_peak,
                     "unit": "TFLOP/s", "frac": dom["tflops"] / fp8_peak,
                     "peak_source": f"{peak_kind} bf16 sustained x {FP8_PER_BF16:g} (nominal fp8:bf16)",
-                    "frac_of_spec_fp8_4500": dom["tflops"] / FP8_DENSE_SPEC_TFLOPS}
+                    "frac_of_spec_fp8_4500": dom["tflops"] / FP8_DENSE_SPEC_TFLOPS,
+                    "frac_of": roofline_fracs(dom["tflops"], pk, peak_kind, ceiling)}
     else:
         roofline = {"bound": "hbm", "kernel": dom_kind, "achieved": dom["gbs"], "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": dom["gbs"] / pk["hbm_gbs"], "peak_source": peak_kind}
@@ -606,7 +673,12 @@ def main_ours(args, rank, world, local_rank):
             "kernels": {k: {"launches": d["launches"], "share": round(d["share"], 4),
                             "avg_us": round(d["avg_us"], 2),
                             "tflops": None if d["tflops"] is None else round(d["tflops"], 1),
-                            "gbs": round(d["gbs"], 1)} for k, d in kinds.items()},
+                            "gbs": round(d["gbs"], 1),
+                            **({"frac_of": {f: round(v, 4) for f, v in
+                                            roofline_fracs(d["tflops"], pk, peak_kind, ceiling).items()}}
+                               if d["tflops"] else {})}
+                        for k, d in kinds.items()},
+            "fp8_library_tflops": ceiling,
             "roofline": roofline,
             "roofline_quantize": roofline_quant,
             "cpu_baseline": cpu,
@@ -720,6 +792,14 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        # one process per GPU: N > 1 is launched by torchrun, which sets
+        # WORLD_SIZE; anything else would time a different number of replicas
+        # than the line reports
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch N > 1 GPUs with "
+              f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus}",
+              file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args, rank)
     return main_ours(args, rank, world, local_rank)

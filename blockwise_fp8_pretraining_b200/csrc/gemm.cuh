@@ -133,14 +133,6 @@ struct Bars {
     __device__ __forceinline__ uint32_t sempty_(int s) const { return sempty + 8 * s; }
 };
 
-// Wait without the abort check, used only while draining after a time-out.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > limit_ns) return;
-    }
-}
-
 template <int SCALE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -226,16 +218,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     ++it;
                 }
             }
-            if (!ok) {
-                // Let every copy already requested land before the pair exits.
-                if (rank == 0) {
-                    for (int j = max(0, it - STAGES); j < it; ++j)
-                        drain_wait(bars.full_(j % STAGES), (j / STAGES) & 1, p.wait_ns);
-                } else {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (globaltimer_ns() - t0 < 200000ull) {
-                    }
-                }
+            if (!ok && rank == 0) {
+                // Let every copy already requested land before the pair
+                // exits.  Both CTAs' copies complete on the leader's full
+                // barriers, so the leader's drain covers rank 1's too, and
+                // rank 1 leaves only after the closing cluster barrier.
+                for (int j = max(0, it - STAGES); j < it; ++j)
+                    drain_wait(bars.full_(j % STAGES), (j / STAGES) & 1, p.wait_ns);
             }
         }
       } else if (warp == 2) {

@@ -429,12 +429,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
             // let loads already requested land before the block exits
             for (int j = 0; j < 2; ++j) {
                 const int64_t tl = blockIdx.x + static_cast<int64_t>(i + j) * gridDim.x;
-                if (tl < total) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(bar0 + 8 * ((i + j) & 1), ((i + j) >> 1) & 1)) {
-                        if (globaltimer_ns() - t0 > wait_ns) break;
-                    }
-                }
+                if (tl < total) drain_wait(bar0 + 8 * ((i + j) & 1), ((i + j) >> 1) & 1, wait_ns);
             }
         }
         bulk_wait_group0();

@@ -94,14 +94,24 @@ def check_weight(w: torch.Tensor):
 # ---------------------------------------------------------------------- GEMMs
 
 def pick_rows(total: int, count: int, seed: int) -> np.ndarray:
-    """Seeded sample of output rows that always includes the first and last
-    row of the first and last 128-row tile."""
+    """Seeded sample of output rows, stratified: one row drawn from every
+    128-row block (so every M tile of the persistent schedule, both CTAs of
+    every pair and the partial last wave are hit), plus the first and last
+    row of the first and last block, plus further seeded rows up to `count`.
+    All rows when count >= total."""
     if count >= total:
         return np.arange(total)
     rng = np.random.default_rng(seed)
+    blocks = (total + 127) // 128
+    strat = np.array([min(total - 1, 128 * b + int(rng.integers(0, 128))) for b in range(blocks)])
     fixed = np.array(sorted({0, min(127, total - 1), max(0, total - 128), total - 1}))
-    rest = rng.choice(total, size=max(0, count - fixed.size), replace=False)
-    return np.unique(np.concatenate([fixed, rest]))
+    rows = np.unique(np.concatenate([fixed, strat]))
+    extra = max(0, count - rows.size)
+    if extra:
+        rest = rng.choice(np.setdiff1d(np.arange(total), rows), size=min(extra, total - rows.size),
+                          replace=False)
+        rows = np.unique(np.concatenate([rows, rest]))
+    return rows
 
 
 def check_fprop(x: torch.Tensor, w: torch.Tensor, rows=None, what="fprop", output_rounding=False):

@@ -164,3 +164,25 @@ def test_clock_rejects_follows_the_timing_rules():
     assert bench.clock_rejects({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})
     # no sampler: nothing to judge by
     assert not bench.clock_rejects({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]})
+
+
+def test_gpus_must_match_the_launched_world_size(monkeypatch, capsys):
+    """--gpus N > 1 without torchrun would time one replica while claiming N:
+    both arms refuse it before doing any work."""
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    for impl in ("ours", "reference"):
+        monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "2", "--impl", impl])
+        assert bench.main() == 2
+        assert "WORLD_SIZE=1" in capsys.readouterr().err
+
+
+def test_roofline_fractions_use_every_denominator():
+    pk = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    ceiling = {"8192x8192x8192": {"tflops": 3000.0}, "gate_up_fprop_8192x12288x2048": {"tflops": 2500.0}}
+    fr = bench.roofline_fracs(1500.0, pk, "measured", ceiling)
+    assert fr["spec_fp8_dense_4500"] == pytest.approx(1500.0 / 4500.0)
+    assert fr["2x_measured_bf16_burst"] == pytest.approx(1500.0 / 3200.0)
+    assert fr["2x_measured_bf16_sustained"] == pytest.approx(1500.0 / 2800.0)
+    assert fr["fp8_library_8192x8192x8192"] == pytest.approx(0.5)
+    assert fr["fp8_library_gate_up_fprop_8192x12288x2048"] == pytest.approx(0.6)
+    assert "fp8_library_8192x8192x8192" not in bench.roofline_fracs(1.0, pk, "measured", {"error": "x"})

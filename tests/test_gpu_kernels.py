@@ -177,7 +177,7 @@ def test_tiny_config_fprop_dgrad_wgrad_full():
     check_weight(c["w"])
     check_fprop(c["x"], c["w"])
     check_dgrad(c["dy"], c["w"])
-    check_wgrad(c["dy"], c["x"], rows=pick_rows(2048, 256, 1))
+    check_wgrad(c["dy"], c["x"])
 
 
 def test_gemm_degenerate_inputs():
