@@ -70,12 +70,6 @@ LAYERS = 28
 # Valid only for the kernels they were taken on; the profiles/ summaries give
 # the commands.  Remove an entry when its kernel changes.
 NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
-    "gemm_rowblock": (46.687e6 + 157.323e6,
-                      "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernels of commit 5a9b046"),
-    "gemm_outer": (122.955e6 + 37.761e6,
-                   "gate_up wgrad 12288x2048x8192 (algorithmic 167.8 MB); kernels of commit 5a9b046"),
-    "quant_act": (201.473e6 + 160.166e6,
-                  "gate_up gradient 8192x12288, both layouts (algorithmic 409 MB); kernels of commit 5a9b046"),
 }
 
 

@@ -15,6 +15,7 @@ from ._abi import (  # noqa: F401
     fp8_block_gemm_dgrad,
     fp8_block_gemm_fprop,
     fp8_block_gemm_wgrad,
+    fp8_block_gemm_wgrad_accum_f32,
     fp8_cast_e4m3_scaled,
     fp8_clear_error,
     fp8_get_error,
@@ -22,6 +23,7 @@ from ._abi import (  # noqa: F401
     fp8_quantize_act_1x128,
     fp8_quantize_weight_128x128,
     fp8_selftest_division,
+    fp8_selftest_stall_next,
     fp8_selftest_wait_timeout,
     fp8_set_wait_timeout_ns,
     fp8_status_string,

@@ -59,11 +59,13 @@ def load() -> ctypes.CDLL:
         "fp8_block_gemm_fprop": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p],
+        "fp8_block_gemm_wgrad_accum_f32": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_get_error": [],
         "fp8_clear_error": [],
         "fp8_set_wait_timeout_ns": [ctypes.c_uint64],
         "fp8_cast_e4m3_scaled": [p, ctypes.c_float, p, i64, p],
         "fp8_selftest_wait_timeout": [p],
+        "fp8_selftest_stall_next": [i32],
         "fp8_selftest_division": [p, p],
     }
     for name, args in sig.items():
@@ -262,6 +264,25 @@ def fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=None, stream=None):
     return dw
 
 
+def fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, stream=None):
+    """dW[N, K] += dY^T X in FP32, in place, from the same along-token codes
+    as fp8_block_gemm_wgrad; dw is a float32 [N, K] tensor (the main
+    gradient).  Returns dw."""
+    lib = load()
+    N, M = dyqT.shape
+    K = xqT.shape[0]
+    _want(dyqT, torch.uint8, (N, M), "dyqT")
+    _want(sdyT, torch.float32, (M // 128, N), "sdyT")
+    _want(xqT, torch.uint8, (K, M), "xqT")
+    _want(sxT, torch.float32, (M // 128, K), "sxT")
+    _want(dw, torch.float32, (N, K), "dw")
+    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw)], stream)
+    _check(lib.fp8_block_gemm_wgrad_accum_f32(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw),
+                                              N, K, M, _stream(stream)),
+           "fp8_block_gemm_wgrad_accum_f32")
+    return dw
+
+
 def fp8_get_error() -> int:
     return int(load().fp8_get_error())
 
@@ -310,3 +331,9 @@ def fp8_selftest_division(stream=None):
 
 def fp8_selftest_wait_timeout(stream=None) -> None:
     _check(load().fp8_selftest_wait_timeout(_stream(stream)), "fp8_selftest_wait_timeout")
+
+
+def fp8_selftest_stall_next(which: int) -> None:
+    """Arm the next GEMM (1), tile quantizer (2) or both (3) launches to run
+    into their bounded wait (test support)."""
+    _check(load().fp8_selftest_stall_next(int(which)), "fp8_selftest_stall_next")

@@ -44,10 +44,19 @@ using namespace fp8blk;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 
+// Test only (fp8_selftest_stall_next): bit 0 arms the next GEMM launch,
+// bit 1 the next tile-quantizer launch, to over-state one barrier's bytes.
+std::atomic<int> g_stall_next{0};
+constexpr uint32_t kStallBytes = 16;
+
+inline uint32_t take_stall(int bit) {
+    return (g_stall_next.fetch_and(~bit) & bit) ? kStallBytes : 0u;
+}
+
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_gemm_attr_done[kMaxDevices];
-std::atomic<int> g_gemm_pairs[kMaxDevices][2];   // co-resident CTA pairs per kernel
+std::atomic<int> g_gemm_pairs[kMaxDevices][4];   // co-resident CTA pairs per kernel variant
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
@@ -120,17 +129,19 @@ fp8_status make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows,
     return FP8_OK;
 }
 
-// Row-major [rows, cols] bf16 output, boxes of 32 rows x 64 columns (128
-// bytes) in the 128-byte swizzle the epilogue's staging buffers use.
-fp8_status make_output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
+// Row-major [rows, cols] GEMM output, boxes of 32 rows x 128 bytes (64 BF16
+// or 32 FP32 columns) in the 128-byte swizzle of the epilogue's staging
+// buffers.
+fp8_status make_output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols, bool f32) {
     auto enc = tensor_map_encoder();
     if (!enc) return FP8_ERR_CUDA;
+    const int esize = f32 ? 4 : 2;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {64u, 32u};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esize};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
     cuuint32_t estride[2] = {1u, 1u};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estride,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+                     strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled(output): CUresult %d", static_cast<int>(r));
@@ -195,23 +206,25 @@ fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t*
     const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
     const cudaError_t e = launch_pdl(quant_tile_kernel<MODE>, dim3(grid), dim3(tile::THREADS), tile::SMEM_BYTES,
                                      stream, mx, mq, mqt, rows, cols, s_row, s_col, qT != nullptr ? 1 : 0,
-                                     g_wait_ns.load(std::memory_order_relaxed));
+                                     g_wait_ns.load(std::memory_order_relaxed), take_stall(2));
     if (e != cudaSuccess) return cuda_fail("tile quantize launch", e);
     return last_launch_status("tile quantize launch");
 }
 
-// Shared launcher of the three GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
-// codes, both K-major; scales described by `p`.
-template <int SCALE>
-fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, gemm::Params p, cudaStream_t stream) {
+// Shared launcher of the GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
+// codes, both K-major; scales described by `p`; out: [M_out, N_out] BF16, or
+// FP32 added to in place (OUT == kOutAccF32).
+template <int SCALE, int OUT>
+fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Params p, cudaStream_t stream) {
     int dev = 0, sms = 0;
     fp8_status st = current_device(&dev);
     if (st != FP8_OK) return st;
     if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
 
-    const int flag = 1 << SCALE;
+    constexpr int variant = SCALE + 2 * OUT;
+    const int flag = 1 << variant;
     if ((g_gemm_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE>,
+        cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE, OUT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              gemm::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
@@ -222,28 +235,42 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, gemm::Params p, cudaS
         cfg.blockDim = dim3(gemm::THREADS, 1, 1);
         cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
         int pairs = 0;
-        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<SCALE>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<SCALE, OUT>, &cfg);
         if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
         if (pairs <= 0) return cuda_fail("gemm kernel cannot be resident", cudaErrorInvalidConfiguration);
-        g_gemm_pairs[dev][SCALE].store(pairs, std::memory_order_relaxed);
+        g_gemm_pairs[dev][variant].store(pairs, std::memory_order_relaxed);
         g_gemm_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
     }
-    const int max_pairs = g_gemm_pairs[dev][SCALE].load(std::memory_order_relaxed);
+    const int max_pairs = g_gemm_pairs[dev][variant].load(std::memory_order_relaxed);
 
     CUtensorMap ma, mb, mc;
     if ((st = make_operand_map(&ma, a, p.M, p.K, gemm::BM)) != FP8_OK) return st;
-    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN / 2)) != FP8_OK) return st;
-    if ((st = make_output_map(&mc, p.out, p.M, p.N)) != FP8_OK) return st;
+    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::B_ROWS)) != FP8_OK) return st;
+    if ((st = make_output_map(&mc, out, p.M, p.N, OUT == gemm::kOutAccF32)) != FP8_OK) return st;
 
     p.tiles_m = static_cast<int>((p.M + 2 * gemm::BM - 1) / (2 * gemm::BM));
     p.tiles_n = static_cast<int>((p.N + gemm::BN - 1) / gemm::BN);
     p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    p.stall_tx = take_stall(1);
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     const int grid = 2 * static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-    const cudaError_t e = launch_pdl(gemm::gemm_kernel<SCALE>, dim3(grid), dim3(gemm::THREADS), gemm::SMEM_BYTES,
-                                     stream, ma, mb, mc, p);
+    const cudaError_t e = launch_pdl(gemm::gemm_kernel<SCALE, OUT>, dim3(grid), dim3(gemm::THREADS),
+                                     gemm::SMEM_BYTES, stream, ma, mb, mc, p);
     if (e != cudaSuccess) return cuda_fail("gemm launch", e);
     return last_launch_status("gemm launch");
+}
+
+// wgrad: dW [N, K] over M tokens; A = dY^T codes [N, M], B = X^T codes [K, M].
+gemm::Params wgrad_params(const float* sdyT, const float* sxT, int64_t N, int64_t K, int64_t M) {
+    gemm::Params p{};
+    p.sa = sdyT;
+    p.sa_ld = N;                 // sdyT [M/128, N]
+    p.sb = sxT;
+    p.sb_ld = K;                 // sxT [M/128, K]
+    p.M = static_cast<int>(N);
+    p.N = static_cast<int>(K);
+    p.K = static_cast<int>(M);
+    return p;
 }
 
 bool dims_ok_gemm(int64_t M, int64_t N, int64_t K, bool m_positive) {
@@ -251,7 +278,7 @@ bool dims_ok_gemm(int64_t M, int64_t N, int64_t K, bool m_positive) {
     if (m_positive && M == 0) return false;
     if (M % 128 || N % 128 || K % 128) return false;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return false;
-    if (static_cast<int64_t>((M + 127) / 128) * ((N + 255) / 256) > kMaxDim) return false;
+    if (static_cast<int64_t>((M + 255) / 256) * ((N + 191) / 192) > kMaxDim) return false;
     return true;
 }
 
@@ -324,11 +351,10 @@ fp8_status fp8_block_gemm_fprop(const uint8_t* xq, const float* sx, const uint8_
     p.sb = sw;
     p.sb_sn = K / 128;           // sw [N/128, K/128]
     p.sb_sk = 1;
-    p.out = static_cast<__nv_bfloat16*>(y_bf16);
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
-    return launch_gemm<gemm::kScaleRowBlock>(xq, wq, p, static_cast<cudaStream_t>(stream));
+    return launch_gemm<gemm::kScaleRowBlock, gemm::kOutBf16>(xq, wq, y_bf16, p, static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_dgrad(const uint8_t* dyq, const float* sdy, const uint8_t* wqT,
@@ -345,11 +371,10 @@ fp8_status fp8_block_gemm_dgrad(const uint8_t* dyq, const float* sdy, const uint
     p.sb = sw;                   // s_b(output block kb, slab nb) = sw[nb][kb]
     p.sb_sn = 1;
     p.sb_sk = K / 128;
-    p.out = static_cast<__nv_bfloat16*>(dx_bf16);
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(K);
     p.K = static_cast<int>(N);
-    return launch_gemm<gemm::kScaleRowBlock>(dyq, wqT, p, static_cast<cudaStream_t>(stream));
+    return launch_gemm<gemm::kScaleRowBlock, gemm::kOutBf16>(dyq, wqT, dx_bf16, p, static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_wgrad(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
@@ -359,16 +384,19 @@ fp8_status fp8_block_gemm_wgrad(const uint8_t* dyqT, const float* sdyT, const ui
     if (!dyqT || !sdyT || !xqT || !sxT || !dw_bf16) return FP8_ERR_NULL;
     if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_bf16))
         return FP8_ERR_ALIGN;
-    gemm::Params p{};
-    p.sa = sdyT;
-    p.sa_ld = N;                 // sdyT [M/128, N]
-    p.sb = sxT;
-    p.sb_ld = K;                 // sxT [M/128, K]
-    p.out = static_cast<__nv_bfloat16*>(dw_bf16);
-    p.M = static_cast<int>(N);
-    p.N = static_cast<int>(K);
-    p.K = static_cast<int>(M);
-    return launch_gemm<gemm::kScaleOuter>(dyqT, xqT, p, static_cast<cudaStream_t>(stream));
+    return launch_gemm<gemm::kScaleOuter, gemm::kOutBf16>(dyqT, xqT, dw_bf16, wgrad_params(sdyT, sxT, N, K, M),
+                                                          static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
+                                          const float* sxT, float* dw_f32, int64_t N, int64_t K, int64_t M,
+                                          void* stream) {
+    if (!dims_ok_gemm(N, K, M, true)) return FP8_ERR_SHAPE;
+    if (!dyqT || !sdyT || !xqT || !sxT || !dw_f32) return FP8_ERR_NULL;
+    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_f32))
+        return FP8_ERR_ALIGN;
+    return launch_gemm<gemm::kScaleOuter, gemm::kOutAccF32>(dyqT, xqT, dw_f32, wgrad_params(sdyT, sxT, N, K, M),
+                                                            static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_get_error(void) {
@@ -425,6 +453,12 @@ fp8_status fp8_selftest_division(unsigned long long* result, void* stream) {
     if (!aligned16(result)) return FP8_ERR_ALIGN;
     division_selftest_kernel<<<0x7F7F, 256, 0, static_cast<cudaStream_t>(stream)>>>(result);
     return last_launch_status("division self-test launch");
+}
+
+fp8_status fp8_selftest_stall_next(int which) {
+    if (which < 1 || which > 3) return FP8_ERR_MODE;
+    g_stall_next.fetch_or(which);
+    return FP8_OK;
 }
 
 fp8_status fp8_selftest_wait_timeout(void* stream) {

@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
     quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmQT, int64_t rows, int64_t cols,
                       float* __restrict__ s_row, float* __restrict__ s_col, int has_qT,
-                      uint64_t wait_ns) {
+                      uint64_t wait_ns, uint32_t stall_tx) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -231,11 +231,13 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
     const bool want_rows = (MODE != kTileColwise);
     const bool want_cols = (MODE != kTileWeight) || has_qT;
 
+    // stall_tx (test only, 0 normally): extra bytes the block's first load
+    // barrier expects, so that its wait runs out
     auto issue_load = [&](int64_t tl, int j) {
         const uint32_t dst = sbase + (j ? tile::OFF_IN1 : tile::OFF_IN0);
         const int32_t x = static_cast<int32_t>((tl % tiles_c) * kGroup);
         const int32_t y = static_cast<int32_t>((tl / tiles_c) * kGroup);
-        mbar_arrive_expect_tx(bar0 + 8 * j, tile::IN_BYTES);
+        mbar_arrive_expect_tx(bar0 + 8 * j, tile::IN_BYTES + (tl == blockIdx.x ? stall_tx : 0u));
         tma_load_2d(dst, &tmX, x, y, bar0 + 8 * j);
         tma_load_2d(dst + tile::BOX_BYTES, &tmX, x + 64, y, bar0 + 8 * j);
     };

@@ -46,10 +46,14 @@
  * failed check returns its status and enqueues nothing.  FP8_ERR_CUDA
  * reports a failed launch (cudaGetLastError after the launch).  Faults that
  * happen later on the device surface at the caller's next synchronization,
- * as with any CUDA work.  Every wait inside a kernel is bounded in time; a
- * wait that runs out makes the kernel record FP8_ERR_TIMEOUT in a sticky
- * per-device error word (read it with fp8_get_error) and return without
- * completing its output.
+ * as with any CUDA work.  Every barrier wait inside a kernel is bounded in
+ * time; a wait that runs out makes the kernel record FP8_ERR_TIMEOUT in a
+ * sticky per-device error word (read it with fp8_get_error) and return
+ * without completing its output.  Before it returns, a kernel still waits
+ * (at most max(limit, 100 ms) per wait) for the copies and tensor-core
+ * operations it has already issued.  The GEMM's two CTAs then meet at one
+ * closing cluster barrier, which has no time limit of its own: both reach it
+ * because every wait before it is bounded.
  */
 #ifndef FP8BLK_H
 #define FP8BLK_H
@@ -86,6 +90,9 @@ enum {
  * Activation quantizer, 1x128 groups (row-wise) and/or 128x1 groups along
  * tokens (column-wise).  Row-wise groups serve fprop (X) and dgrad (dY);
  * column-wise groups serve wgrad, which contracts over tokens.
+ * Passage: Puro-2B-Base model card (friendli.ai), training-setup paragraph
+ * ("blockwise E4M3" linear-layer GEMMs); group shape and scale as defined at
+ * the top of this header.
  *
  *   x_bf16  [rows, cols] bf16, 16-byte aligned.
  *   rows    >= 0; a multiple of 128 when mode includes FP8_COLWISE.
@@ -104,6 +111,9 @@ fp8_status fp8_quantize_act_1x128(const void *x_bf16, int64_t rows, int64_t cols
 
 /*
  * Weight quantizer, 128x128 blocks.
+ * Passage: Puro-2B-Base model card, training-setup paragraph (blockwise E4M3);
+ * the 128x128 block follows the DeepSeek-V3 recipe the Puro-2B tech report
+ * cites (part 7/7, section 5).
  *
  *   w_bf16  [n, k] bf16, 16-byte aligned; n, k >= 0, multiples of 128.
  *   wq      [n, k] u8 codes.
@@ -118,6 +128,9 @@ fp8_status fp8_quantize_weight_128x128(const void *w_bf16, int64_t n, int64_t k,
 
 /*
  * fprop: Y[m, n] = sum_k X[m, k] W[n, k]   (Y = X W^T), BF16 out.
+ * Passage: Puro-2B-Base model card, training-setup paragraph (the main
+ * linear-layer GEMMs run in blockwise E4M3, other tensors in BF16); per-slab
+ * FP32 promotion after the DeepSeek-V3 recipe (tech report part 7/7, sec. 5).
  *
  *   xq [M, K] u8, sx [K/128, M] f32   - row-wise quantized X
  *   wq [N, K] u8, sw [N/128, K/128] f32 - 128x128 quantized W
@@ -132,6 +145,10 @@ fp8_status fp8_block_gemm_fprop(const uint8_t *xq, const float *sx, const uint8_
 
 /*
  * dgrad: dX[m, k] = sum_n dY[m, n] W[n, k]   (dX = dY W), BF16 out.
+ * Passage: as fprop (model card, training-setup paragraph; tech report part
+ * 7/7, section 5).  The weight operand is the transposed copy of the codes,
+ * which the weight quantizer writes beside the row-major ones, so that the
+ * contraction over n runs along contiguous bytes.
  *
  *   dyq [M, N] u8, sdy [N/128, M] f32 - row-wise quantized dY (groups run
  *                                        along n, the contraction)
@@ -151,6 +168,10 @@ fp8_status fp8_block_gemm_dgrad(const uint8_t *dyq, const float *sdy, const uint
 /*
  * wgrad: dW[n, k] = sum_m dY[m, n] X[m, k]   (dW = dY^T X), contracting over
  * the M tokens, BF16 out.
+ * Passage: as fprop (model card, training-setup paragraph; tech report part
+ * 7/7, section 5).  Both operands are grouped along the tokens, so the
+ * promotion coefficient of a slab is the outer product of the two scale
+ * vectors.
  *
  *   dyqT [N, M] u8, sdyT [M/128, N] f32 - column-wise (along-token) dY
  *   xqT  [K, M] u8, sxT  [M/128, K] f32 - column-wise (along-token) X
@@ -160,6 +181,26 @@ fp8_status fp8_block_gemm_dgrad(const uint8_t *dyq, const float *sdy, const uint
 fp8_status fp8_block_gemm_wgrad(const uint8_t *dyqT, const float *sdyT, const uint8_t *xqT,
                                 const float *sxT, void *dw_bf16, int64_t N, int64_t K,
                                 int64_t M, void *stream);
+
+/*
+ * wgrad accumulated into an FP32 main gradient: dW_f32[n, k] += sum_m
+ * dY[m, n] X[m, k], with the same operands, promotion and error bound as
+ * fp8_block_gemm_wgrad.  Each output element receives one FP32 addition
+ * (round-to-nearest-even) of this call's FP32 result to the value in memory,
+ * so successive micro-batches accumulate in place without a BF16 rounding.
+ * Passage: Puro-2B-Base model card, training-setup paragraph (master weights
+ * and optimizer state stay in FP32); the accumulation over the micro-batches
+ * of one optimizer step follows from the setting table (global batch 1536,
+ * micro-batch 2).
+ *
+ *   dyqT, sdyT, xqT, sxT, N, K, M - as fp8_block_gemm_wgrad
+ *   dw_f32 [N, K] f32, read and written (16-byte aligned); must not overlap
+ *          the inputs.  Calls on the same dw_f32 must be ordered (one stream).
+ */
+fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t *dyqT, const float *sdyT,
+                                          const uint8_t *xqT, const float *sxT,
+                                          float *dw_f32, int64_t N, int64_t K, int64_t M,
+                                          void *stream);
 
 /* Sticky per-device error word: FP8_OK, or the first FP8_ERR_TIMEOUT a
  * kernel recorded on the current device since the last clear.  Reading it
@@ -204,6 +245,17 @@ fp8_status fp8_selftest_division(unsigned long long *result, void *stream);
  * records FP8_ERR_TIMEOUT in the sticky error word.  For testing the timeout
  * path; nothing else is touched. */
 fp8_status fp8_selftest_wait_timeout(void *stream);
+
+/* Arms the next launch of a kernel family so that the first operand
+ * barrier of every CTA (pair) expects 16 bytes more than its copies bring:
+ * that wait runs out after the current time limit, the kernel
+ * records FP8_ERR_TIMEOUT, drains what it issued and returns without
+ * completing its output.  which: 1 = the next GEMM launch, 2 = the next
+ * 128x128 tile quantizer launch (column-wise, both layouts or weights),
+ * 3 = both.  Host-side flag shared by all threads and devices; each armed
+ * family is disarmed by its next launch.  For testing the time-out path of
+ * the real kernels; FP8_ERR_MODE for any other value. */
+fp8_status fp8_selftest_stall_next(int which);
 
 #ifdef __cplusplus
 }

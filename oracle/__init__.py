@@ -65,6 +65,8 @@ def _configure(lib: ctypes.CDLL) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p]
+    lib.orc_gemm_wgrad_accum.restype = ctypes.c_int
+    lib.orc_gemm_wgrad_accum.argtypes = [p, p, p, p, i64, i64, i64, p, i64, p, p, p]
     lib.orc_num_threads.restype = ctypes.c_int
     lib.orc_num_threads.argtypes = []
     lib.orc_bf16_from_double.restype = ctypes.c_uint16
@@ -242,6 +244,29 @@ def gemm_wgrad(dyqT, sdyT, xqT, sxT, rows=None):
     _check(_load().orc_gemm_wgrad(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), N, K, M,
                                   None if r is None else _ptr(r), nr, _ptr(y), _ptr(b)),
            "gemm_wgrad")
+    return y, b
+
+
+def gemm_wgrad_accum(dyqT, sdyT, xqT, sxT, dw_in=None, rows=None):
+    """Main-gradient accumulation: dw_in + dY^T X in FP64 on the selected
+    output rows.  dw_in float64 [N, K] (the running main gradient; an FP32
+    array converts exactly) or None for zeros.  Returns (dw, bound) float64
+    [len(rows) or N, K]; bound is this call's wgrad bound."""
+    dyqT = _c(dyqT, np.uint8); sdyT = _c(sdyT, np.float32)
+    xqT = _c(xqT, np.uint8); sxT = _c(sxT, np.float32)
+    N, M = dyqT.shape
+    K = xqT.shape[0]
+    assert xqT.shape[1] == M and sdyT.shape == (M // GROUP, N) and sxT.shape == (M // GROUP, K)
+    if dw_in is not None:
+        dw_in = _c(dw_in, np.float64)
+        assert dw_in.shape == (N, K)
+    r, nr = _rows_arg(rows, N)
+    y = np.empty((nr, K), np.float64)
+    b = np.empty((nr, K), np.float64)
+    _check(_load().orc_gemm_wgrad_accum(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), N, K, M,
+                                        None if r is None else _ptr(r), nr,
+                                        None if dw_in is None else _ptr(dw_in), _ptr(y), _ptr(b)),
+           "gemm_wgrad_accum")
     return y, b
 
 

@@ -403,6 +403,42 @@ int orc_gemm_wgrad(const uint8_t *dyqT, const float *sdyT, const uint8_t *xqT,
     return 0;
 }
 
+/* wgrad accumulated into a main gradient kept across micro-batches: the
+ * Puro-2B-Base model card (friendli.ai), training-setup paragraph, keeps
+ * master weights and optimizer state in FP32, and one optimizer step sums
+ * the weight gradients of its micro-batches (setting table: global batch
+ * 1536 sequences, micro-batch 2).  dw_out[i, k] = dw_in[n, k] + dW[n, k]
+ * for output row n = rows[i] (all rows when rows is NULL), with dW exactly
+ * as orc_gemm_wgrad computes it and the sum taken in FP64.  dw_in is the
+ * running main gradient [N, K] in FP64 (an FP32 array converts to it
+ * exactly; NULL means zeros), so chained calls accumulate without rounding
+ * to FP32 in between.  bound is the wgrad bound of this call's product. */
+int orc_gemm_wgrad_accum(const uint8_t *dyqT, const float *sdyT,
+                         const uint8_t *xqT, const float *sxT, int64_t N,
+                         int64_t K, int64_t M, const int64_t *rows,
+                         int64_t nrows, const double *dw_in, double *dw_out,
+                         double *bound)
+{
+    int rc = orc_gemm_wgrad(dyqT, sdyT, xqT, sxT, N, K, M, rows, nrows,
+                            dw_out, bound);
+    if (rc != 0)
+        return rc;
+    if (!dw_in)
+        return 0;
+    if (!rows)
+        nrows = N;
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t n = rows ? rows[i] : i;
+        for (int64_t k = 0; k < K; ++k) {
+            double v = dw_in[n * K + k];
+            if (!isfinite(v))
+                return -2;
+            dw_out[i * K + k] = v + dw_out[i * K + k];
+        }
+    }
+    return 0;
+}
+
 /* Threads the parallel loops above use. */
 int orc_num_threads(void)
 {

@@ -160,3 +160,16 @@ def test_plain_c_client_compiles_links_and_gets_host_statuses(lib, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
     assert r.stdout.strip() == "ok"
+
+
+def test_stall_switch_rejects_unknown_kernel_families(lib):
+    for bad in (0, 4, -1):
+        assert lib.fp8_selftest_stall_next(bad) == MODE
+
+
+def test_wgrad_accum_rejections(lib):
+    g = lib.fp8_block_gemm_wgrad_accum_f32
+    assert g(P(A16), P(A16), P(A16), P(A16), P(A16), 128, 128, 0, S) == SHAPE      # no tokens
+    assert g(P(A16), P(A16), P(A16), P(A16), P(A16), 128, 100, 128, S) == SHAPE
+    assert g(P(A16), P(A16), P(A16), P(A16), None, 128, 128, 128, S) == NULL
+    assert g(P(A16), P(A16), P(A16), P(A16), P(MIS), 128, 128, 128, S) == ALIGN

@@ -1,6 +1,6 @@
 """GPU parity of every kernel against the CPU oracle at sizes the oracle
 finishes in seconds: several tiles, ragged tails (row counts that are not a
-multiple of a block's rows, N = 128 * odd against 256-wide GEMM tiles, grids
+multiple of a block's rows, N against 192-wide GEMM pair tiles, grids
 with fewer tiles than SMs and with a partial last wave), heavy tails, zero
 groups, and the degenerate cases of the method."""
 import numpy as np
@@ -11,8 +11,8 @@ import blockwise_fp8_pretraining_b200 as fp8
 import oracle
 from blockwise_fp8_pretraining_b200 import synthetic as syn
 
-from _parity import (assert_bits_equal, check_act, check_dgrad, check_fprop, check_wgrad,
-                     check_weight, dev, pick_rows)
+from _parity import (assert_bits_equal, assert_within_bound, check_act, check_dgrad, check_fprop,
+                     check_wgrad, check_weight, dev, pick_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -246,3 +246,137 @@ def test_bounded_wait_times_out_and_reports():
     # the context is still usable afterwards
     check_fprop(syn.normal_bf16((128, 128), 1.0, syn.generator(1)),
                 syn.normal_bf16((128, 128), 0.02, syn.generator(2)))
+
+
+# ------------------------------------------------------------ guard bands
+
+GUARD_ROWS = 3
+
+
+def _guarded(rows, cols, dtype, fill_bits):
+    """A [rows, cols] view in the middle of a buffer whose GUARD_ROWS rows
+    before and after are filled with a sentinel bit pattern."""
+    itemsize = torch.empty((), dtype=dtype).element_size()
+    int_t = {2: torch.int16, 4: torch.int32}[itemsize]
+    buf = torch.full((rows + 2 * GUARD_ROWS, cols), fill_bits, dtype=int_t, device=dev()).view(dtype)
+    return buf, buf[GUARD_ROWS:GUARD_ROWS + rows]
+
+
+def _assert_guards(buf, rows, fill_bits, what):
+    int_t = {2: torch.int16, 4: torch.int32}[buf.element_size()]
+    raw = buf.view(int_t)
+    for part, name in ((raw[:GUARD_ROWS], "before"), (raw[GUARD_ROWS + rows:], "after")):
+        bad = int((part != fill_bits).sum())
+        assert bad == 0, f"{what}: {bad} guard elements {name} the output were written"
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (384, 640, 256), (128, 256, 384), (640, 2560, 128)])
+def test_gemm_writes_stay_inside_the_output(M, N, K):
+    """Ragged tiles (N against 192-wide pair tiles, M = 128 against 256-row
+    pair tiles): outputs are views inside sentinel-filled buffers, and every
+    sentinel must survive fprop, dgrad and wgrad."""
+    d = dev()
+    g = syn.generator(M + 3 * N + 7 * K)
+    x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
+    w = syn.normal_bf16((N, K), 0.02, g)
+    dy = syn.normal_bf16((M, N), 1e-3, g)
+    sentinel = 0x7FA5          # a bfloat16 NaN pattern the kernels never produce
+    xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x.to(d), fp8.ROWWISE)
+    wq, sw, wqT = fp8.fp8_quantize_weight_128x128(w.to(d))
+    buf, y = _guarded(M, N, torch.bfloat16, sentinel)
+    fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, y=y)
+    dyq, sdy, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.BOTH)
+    dbuf, dx = _guarded(M, K, torch.bfloat16, sentinel)
+    fp8.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=dx)
+    _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
+    wbuf, dw = _guarded(N, K, torch.bfloat16, sentinel)
+    fp8.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=dw)
+    fbuf, dwf = _guarded(N, K, torch.float32, 0x7FC0A5A5)
+    dwf.zero_()
+    fp8.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dwf)
+    torch.cuda.synchronize()
+    _assert_guards(buf, M, sentinel, "fprop")
+    _assert_guards(dbuf, M, sentinel, "dgrad")
+    _assert_guards(wbuf, N, sentinel, "wgrad")
+    _assert_guards(fbuf, N, 0x7FC0A5A5, "wgrad accumulate")
+    xq_o, sx_o = oracle.quantize_act_rowwise(syn.bf16_bits(x))
+    wq_o, sw_o = oracle.quantize_weight(syn.bf16_bits(w))
+    y_o, b_o = oracle.gemm_fprop(xq_o, sx_o, wq_o, sw_o)
+    assert_within_bound(y, y_o, b_o, "fprop in a guarded buffer", output_rounding=True)
+
+
+# -------------------------------------------- FP32 main-gradient accumulation
+
+def _accumulate(N, K, M, micro_batches, seed, rows=None):
+    """micro_batches wgrad products added into one FP32 main gradient on the
+    GPU, and the same sum in FP64 by the oracle (both starting from the same
+    seeded FP32 values).  Bound: each call's 2e-3 S + 1e-6, plus the FP32
+    rounding of each addition on the GPU (half an ulp of the running value)."""
+    d = dev()
+    dw0 = torch.from_numpy(np.random.default_rng(seed).normal(scale=0.01, size=(N, K)).astype(np.float32))
+    dw = dw0.to(d)
+    running = dw0.numpy().astype(np.float64)
+    tol = np.zeros((N, K) if rows is None else (len(rows), K))
+    for b in range(micro_batches):
+        g = syn.generator(seed * 1000 + b)
+        dy = syn.normal_bf16((M, N), 1e-3, g)
+        x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
+        _, _, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.COLWISE)
+        _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
+        fp8.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw)
+        dyqT_o, sdyT_o = oracle.quantize_act_colwise(syn.bf16_bits(dy))
+        xqT_o, sxT_o = oracle.quantize_act_colwise(syn.bf16_bits(x))
+        new, bound = oracle.gemm_wgrad_accum(dyqT_o, sdyT_o, xqT_o, sxT_o, running)
+        running = new
+        sel = running if rows is None else running[rows]
+        tol += 2e-3 * (bound if rows is None else bound[rows]) + 1e-6 + 2.0 ** -24 * np.abs(sel)
+    torch.cuda.synchronize()
+    got = dw.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got, running = got[rows], running[rows]
+    err = np.abs(got - running)
+    assert np.all(err <= tol), f"{int((err > tol).sum())} elements outside the accumulated bound"
+
+
+@pytest.mark.parametrize("micro_batches", [2, 32])
+def test_wgrad_accumulates_in_fp32_over_micro_batches(micro_batches):
+    _accumulate(384, 640, 256, micro_batches, seed=micro_batches)
+
+
+@pytest.mark.slow
+def test_wgrad_accumulates_in_fp32_at_the_qkv_shape():
+    """Two 8192-token micro-batches into the fused-QKV main gradient
+    [4096, 2048], every element."""
+    _accumulate(syn.QKV_OUT, syn.HIDDEN, syn.TOKENS, 2, seed=5)
+
+
+# ----------------------------------------------- time-outs of the real kernels
+
+def test_gemm_and_quantizer_time_out_drain_and_recover():
+    """An over-stated barrier byte count makes the first operand wait of every
+    CTA run out: the GEMM and the tile quantizer must record FP8_ERR_TIMEOUT,
+    drain what they issued and return, and the next launches must be
+    correct."""
+    d = dev()
+    x = syn.activation_bf16(128, 128, 1, 30.0, syn.generator(41))
+    w = syn.normal_bf16((128, 128), 0.02, syn.generator(42))
+    xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x.to(d), fp8.ROWWISE)
+    wq, sw, _ = fp8.fp8_quantize_weight_128x128(w.to(d), transposed=False)
+    torch.cuda.synchronize()
+    fp8.fp8_clear_error()
+    fp8.fp8_set_wait_timeout_ns(20_000_000)          # 20 ms
+    try:
+        fp8.fp8_selftest_stall_next(1)
+        fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+        assert fp8.fp8_get_error() == 6               # FP8_ERR_TIMEOUT
+        fp8.fp8_clear_error()
+        fp8.fp8_selftest_stall_next(2)
+        fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
+        assert fp8.fp8_get_error() == 6
+        fp8.fp8_clear_error()
+    finally:
+        fp8.fp8_set_wait_timeout_ns(0)
+        fp8.fp8_clear_error()
+    check_fprop(x, w)
+    check_act(x, fp8.COLWISE)
+    assert fp8.fp8_get_error() == 0

@@ -482,6 +482,57 @@ def test_gemm_against_exact_rational_arithmetic():
             assert abs(Fraction(dwb[ri, k]) - exact_abs) <= Fraction(tol)
 
 
+# ------------------------------------------------- main-gradient accumulation
+
+def test_wgrad_accum_all_ones_closed_form_over_two_micro_batches():
+    """dY = X = all-ones over 128 tokens: every along-token code is 0x7E (448)
+    with s = fp32(1/448), so one micro-batch adds exactly 128 (448 s)^2 to
+    every element.  Two micro-batches on a dyadic FP32 starting gradient give
+    v + 2 * 128 (448 s)^2; selected rows read their own starting values."""
+    ones = to_bf16_bits(np.ones((128, 256), np.float32))       # [tokens, N = K = 256]
+    qT, sT = oracle.quantize_act_colwise(ones)                   # [256, 128], [1, 256]
+    assert np.all(qT == 0x7E)
+    s = Fraction(float(np.float32(1.0) / np.float32(448.0)))
+    y = 128 * (448 * s) ** 2
+    n_idx, k_idx = np.meshgrid(np.arange(256), np.arange(256), indexing="ij")
+    v = ((n_idx - 100) * 0.25 + k_idx * 2.0 ** -10).astype(np.float32)
+    rows = [5, 100, 255]
+    out1, b1 = oracle.gemm_wgrad_accum(qT, sT, qT, sT, v.astype(np.float64))
+    out2, _ = oracle.gemm_wgrad_accum(qT, sT, qT, sT, out1)
+    sub, _ = oracle.gemm_wgrad_accum(qT, sT, qT, sT, out1, rows=rows)
+    for n in rows:
+        for k in (0, 1, 77, 255):
+            want = Fraction(float(v[n, k])) + 2 * y
+            assert abs(Fraction(out2[n, k]) - want) <= 2 * Fraction(2) ** -52 * abs(want)
+    assert np.array_equal(sub, out2[rows])
+    assert np.all(np.abs(b1 - float(y)) <= 2.0 ** -52 * float(y))
+    zero, _ = oracle.gemm_wgrad_accum(qT, sT, qT, sT, None)
+    assert np.all(np.abs(zero - float(y)) <= 2.0 ** -52 * float(y))
+
+
+def test_wgrad_accum_against_exact_rational_arithmetic():
+    """A 3-slab wgrad added to a random FP32 running gradient, selected rows,
+    against the exact rational sum dw_in + sum_t sum_m s_a s_b a b."""
+    dyT = syn.normal_bf16((384, 128), 1e-3, syn.generator(31))
+    xT = syn.activation_bf16(384, 256, 2, 30.0, syn.generator(32))
+    dyqT, sdyT = oracle.quantize_act_colwise(syn.bf16_bits(dyT))      # [128, 384]
+    xqT, sxT = oracle.quantize_act_colwise(syn.bf16_bits(xT))         # [256, 384]
+    v = np.random.default_rng(33).normal(scale=0.05, size=(128, 256)).astype(np.float32)
+    rows = [100, 3]
+    dw, _ = oracle.gemm_wgrad_accum(dyqT, sdyT, xqT, sxT, v.astype(np.float64), rows=rows)
+    da, db = torch_decode(dyqT), torch_decode(xqT)
+    for ri, n in enumerate(rows):
+        for k in (0, 130, 255):
+            exact = _exact(v[n, k])
+            exact_abs = abs(exact)
+            for t in range(3):
+                for m in range(t * G, (t + 1) * G):
+                    prod = _exact(sdyT[t, n]) * _exact(da[n, m]) * _exact(sxT[t, k]) * _exact(db[k, m])
+                    exact += prod
+                    exact_abs += abs(prod)
+            assert abs(Fraction(dw[ri, k]) - exact) <= Fraction(8 * 2.0 ** -53 * float(exact_abs))
+
+
 # -------------------------------------------------------------------- SwiGLU
 
 def _bf16_rne_exact(v: Fraction, negative: bool) -> int:

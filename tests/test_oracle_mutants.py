@@ -89,6 +89,12 @@ MUTANTS = [
     ("swiglu: silu not rounded to bfloat16 before the product",
      "double s = (double)orc_bf16_to_float(orc_silu_bf16(gate[j]));",
      "double s = (double)gf / (1.0 + exp(-(double)gf));", None),
+    ("main-gradient accumulation drops the running value",
+     "dw_out[i * K + k] = v + dw_out[i * K + k];", "dw_out[i * K + k] = 0.0 * v + dw_out[i * K + k];", None),
+    ("main-gradient accumulation reads the running value of output position i, not row n",
+     "double v = dw_in[n * K + k];", "double v = dw_in[i * K + k];", None),
+    ("main-gradient accumulation subtracts the product",
+     "dw_out[i * K + k] = v + dw_out[i * K + k];", "dw_out[i * K + k] = v - dw_out[i * K + k];", None),
 ]
 
 
