@@ -88,6 +88,8 @@ def parse():
                     help="--impl reference: oracle work of all warm-up and timed steps together")
     ap.add_argument("--graphs", type=int, default=8, help="distinct captured step graphs")
     ap.add_argument("--no-ceiling", action="store_true", help="skip the FP8 library ceiling measurement")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the per-launch timing of the fused SwiGLU producer and the FP32 main-grad wgrad")
     return ap.parse_args()
 
 
@@ -190,6 +192,38 @@ class Sweep:
             for name, n, k in reversed(shapes):
                 out += self._launches_linear(self.layer[l][name], self.shared[name], name, n, k, "bwd")
         return out
+
+
+def extra_launches(sweep):
+    """Launches of the two kernels outside the step's sweep, on the step's own
+    buffers (after it has run): the fused SwiGLU producer on every layer's
+    gate_up fprop output (H's codes for the down projection without H in
+    memory) and the wgrad of every linear accumulated into FP32 main
+    gradients."""
+    import torch
+
+    T = TOKENS
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    out = []
+    ffn = dict((name, n) for name, n, _ in linear_shapes())["gate_up"] // 2
+    gu, dn = sweep.shared["gate_up"], sweep.shared["down"]
+    for l in range(sweep.layers):
+        per = sweep.layer[l]["down"]
+        out.append(("swiglu_quant_fused", "fp8_swiglu_quantize_1x128",
+                    lambda s, per=per: (P(gu["y"]), T, ffn, 3, P(dn["xq"]), P(dn["sx"]), P(per["xqT"]),
+                                        P(per["sxT"]), s),
+                    0.0, T * ffn * (2 * 2 + 1 + 1 + 8 / 128)))
+    if not hasattr(sweep, "main_grad"):
+        sweep.main_grad = {name: torch.zeros((n, k), dtype=torch.float32, device=sweep.device)
+                           for name, n, k in linear_shapes()}
+    for l in range(sweep.layers):
+        for name, n, k in linear_shapes():
+            sh, per, mg = sweep.shared[name], sweep.layer[l][name], sweep.main_grad[name]
+            out.append(("gemm_outer_accum_f32", "fp8_block_gemm_wgrad_accum_f32",
+                        lambda s, sh=sh, per=per, mg=mg, n=n, k=k: (P(sh["dyqT"]), P(sh["sdyT"]), P(per["xqT"]),
+                                                                   P(per["sxT"]), P(mg), n, k, T, s),
+                        2.0 * T * n * k, T * n + T * k + 2 * 4 * n * k))
+    return out
 
 
 def run_launches(lib, launches, stream_handle, events=None):
@@ -606,6 +640,44 @@ def main_ours(args, rank, world, local_rank):
         e2e_ms = max_over_ranks(e2e.pop("_elapsed_ms"), device, world)
         e2e["value"] = job_tflops(world, flop_step, args.e2e_steps, e2e_ms)
 
+    # ---- kernels outside the step, per launch (after the timed region)
+    extra = None
+    if not args.no_extra:
+        xl = extra_launches(sweep)
+        with torch.cuda.stream(stream):
+            run_launches(lib, xl, stream.cuda_stream)          # warm-up, sets attributes
+        torch.cuda.synchronize()
+        xevents, xgraphs = [], []
+        for _ in range(3):
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(xl) + 1)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run_launches(lib, xl, torch.cuda.current_stream().cuda_stream, evs)
+            xgraphs.append(g)
+            xevents.append(evs)
+        for g in xgraphs:
+            g.replay()
+        torch.cuda.synchronize()
+        xk = summarize_kernels(xl, xevents, pk, peak_kind)
+        for g in xgraphs:
+            g.reset()
+        if fp8.fp8_get_error() != 0:
+            raise RuntimeError("device error word set by the extra kernels")
+        ffn_elems = TOKENS * 6144
+        extra = {k: {"launches": d["launches"], "avg_us": round(d["avg_us"], 2),
+                     "tflops": None if d["tflops"] is None else round(d["tflops"], 1),
+                     "gbs": round(d["gbs"], 1)} for k, d in xk.items()}
+        sq = extra.get("swiglu_quant_fused")
+        if sq:
+            sq["frac_of_hbm"] = round(sq["gbs"] / pk["hbm_gbs"], 4)
+            sq["algorithmic_bytes_per_launch"] = ffn_elems * (4 + 2 + 8 / 128)
+            # an unfused SwiGLU kernel writes H in bf16 and the quantizer reads it back
+            sq["hbm_bytes_saved_per_layer_vs_unfused"] = ffn_elems * 4
+            sq["input"] = "each layer's gate_up fprop output [8192, 12288] (gate | up), both layouts out"
+        oa = extra.get("gemm_outer_accum_f32")
+        if oa:
+            oa["note"] = "wgrad of every linear added into FP32 main gradients (TMA reduce-add epilogue)"
+
     # ---- measured FP8 library ceiling (outside every timed region)
     ceiling = None if args.no_ceiling else fp8_library_ceiling(device)
 
@@ -673,6 +745,7 @@ def main_ours(args, rank, world, local_rank):
                                if d["tflops"] else {})}
                         for k, d in kinds.items()},
             "fp8_library_tflops": ceiling,
+            "kernels_outside_step": extra,
             "roofline": roofline,
             "roofline_quantize": roofline_quant,
             "cpu_baseline": cpu,

@@ -23,10 +23,12 @@ from ._abi import (  # noqa: F401
     fp8_quantize_act_1x128,
     fp8_quantize_weight_128x128,
     fp8_selftest_division,
+    fp8_selftest_silu_bf16,
     fp8_selftest_stall_next,
     fp8_selftest_wait_timeout,
     fp8_set_wait_timeout_ns,
     fp8_status_string,
+    fp8_swiglu_quantize_1x128,
     header_functions,
     lib_path,
     load,

@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
     sig = {
         "fp8_quantize_act_1x128": [p, i64, i64, i32, p, p, p, p, p],
         "fp8_quantize_weight_128x128": [p, i64, i64, p, p, p, p],
+        "fp8_swiglu_quantize_1x128": [p, i64, i64, i32, p, p, p, p, p],
+        "fp8_selftest_silu_bf16": [p, p],
         "fp8_block_gemm_fprop": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p],
@@ -181,6 +183,40 @@ def fp8_quantize_act_1x128(x, mode=BOTH, q_row=None, s_row=None, q_colT=None, s_
                                       _ptr(q_colT), _ptr(s_col), _stream(stream)),
            "fp8_quantize_act_1x128")
     return q_row, s_row, q_colT, s_col
+
+
+def fp8_swiglu_quantize_1x128(gate_up, mode=BOTH, q_row=None, s_row=None, q_colT=None, s_col=None,
+                              stream=None):
+    """Quantize H = silu(gate) * up (bf16 roundings as the unfused path) of
+    a bf16 gate_up activation [rows, 2 * ffn] without forming H in memory.
+    Returns (q_row, s_row, q_colT, s_col) of H [rows, ffn]; entries of a
+    grouping the mode leaves out are None."""
+    lib = load()
+    if gate_up.dtype != torch.bfloat16 or gate_up.dim() != 2 or gate_up.shape[1] % 2:
+        raise TypeError("gate_up must be a 2-D bfloat16 tensor with an even number of columns")
+    rows, cols2 = gate_up.shape
+    ffn = cols2 // 2
+    _want(gate_up, torch.bfloat16, (rows, cols2), "gate_up")
+    dev = gate_up.device
+    given = [t is not None for t in (q_row, s_row, q_colT, s_col)]
+    if mode & ROWWISE:
+        q_row = _out(q_row, torch.uint8, (rows, ffn), dev, "q_row")
+        s_row = _out(s_row, torch.float32, (ffn // 128, rows), dev, "s_row")
+    else:
+        q_row = s_row = None
+    if mode & COLWISE:
+        q_colT = _out(q_colT, torch.uint8, (ffn, rows), dev, "q_colT")
+        s_col = _out(s_col, torch.float32, (rows // 128, ffn), dev, "s_col")
+    else:
+        q_colT = s_col = None
+    outs = (q_row, s_row, q_colT, s_col)
+    _launch_checks([("gate_up", gate_up), ("q_row", q_row), ("s_row", s_row), ("q_colT", q_colT),
+                    ("s_col", s_col)], stream)
+    _record(stream, [t for t, g in zip(outs, given) if not g])
+    _check(lib.fp8_swiglu_quantize_1x128(_ptr(gate_up), rows, ffn, int(mode), _ptr(q_row), _ptr(s_row),
+                                         _ptr(q_colT), _ptr(s_col), _stream(stream)),
+           "fp8_swiglu_quantize_1x128")
+    return outs
 
 
 def fp8_quantize_weight_128x128(w, wq=None, sw=None, wqT=None, transposed=True, stream=None):
@@ -337,3 +373,13 @@ def fp8_selftest_stall_next(which: int) -> None:
     """Arm the next GEMM (1), tile quantizer (2) or both (3) launches to run
     into their bounded wait (test support)."""
     _check(load().fp8_selftest_stall_next(int(which)), "fp8_selftest_stall_next")
+
+
+def fp8_selftest_silu_bf16(stream=None):
+    """silu of every bfloat16 bit pattern as the fused SwiGLU producer
+    computes it: a numpy uint16 array of 65536 bit patterns (index = input
+    bits)."""
+    out = torch.empty(65536, dtype=torch.int16, device="cuda")
+    _check(load().fp8_selftest_silu_bf16(_ptr(out), _stream(stream)), "fp8_selftest_silu_bf16")
+    torch.cuda.synchronize()
+    return out.cpu().numpy().view("uint16")

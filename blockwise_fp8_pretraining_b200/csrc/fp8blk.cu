@@ -172,24 +172,26 @@ fp8_status make_map_2d(CUtensorMap* map, CUtensorMapDataType type, int elem_byte
 
 std::atomic<int> g_tile_attr_done[kMaxDevices];
 
-// Persistent 128 x 128 tile quantizer (column-wise, both, or weight blocks).
-template <int MODE>
+// Persistent 128 x 128 tile quantizer (column-wise, both, weight blocks, or,
+// with SWIGLU, the SwiGLU product of a gate_up activation [rows, 2 * cols]).
+template <int MODE, bool SWIGLU>
 fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* s_row,
                              uint8_t* qT, float* s_col, cudaStream_t stream) {
+    using L = tile::Layout<SWIGLU>;
     int dev = 0, sms = 0;
     fp8_status st = current_device(&dev);
     if (st != FP8_OK) return st;
     if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
-    const int flag = 1 << MODE;
+    const int flag = 1 << (MODE + 4 * (SWIGLU ? 1 : 0));
     if ((g_tile_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
-        const cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE>,
+        const cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE, SWIGLU>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   tile::SMEM_BYTES);
+                                                   L::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(quantize)", e);
         g_tile_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
     }
     CUtensorMap mx, mq, mqt;
-    if ((st = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, rows, cols, 64, 128,
+    if ((st = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, rows, SWIGLU ? 2 * cols : cols, 64, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B, "quantize input")) != FP8_OK)
         return st;
     // Unused maps still need a valid encoding: point them at an output.
@@ -202,11 +204,12 @@ fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t*
                           128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "transposed codes")) != FP8_OK)
         return st;
     const int64_t tiles = (rows / 128) * (cols / 128);
-    const int64_t cap = 2 * static_cast<int64_t>(sms);
+    const int64_t cap = static_cast<int64_t>(L::BLOCKS_PER_SM) * sms;
     const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
-    const cudaError_t e = launch_pdl(quant_tile_kernel<MODE>, dim3(grid), dim3(tile::THREADS), tile::SMEM_BYTES,
-                                     stream, mx, mq, mqt, rows, cols, s_row, s_col, qT != nullptr ? 1 : 0,
-                                     g_wait_ns.load(std::memory_order_relaxed), take_stall(2));
+    const cudaError_t e = launch_pdl(quant_tile_kernel<MODE, SWIGLU>, dim3(grid), dim3(tile::THREADS),
+                                     L::SMEM_BYTES, stream, mx, mq, mqt, rows, cols, s_row, s_col,
+                                     qT != nullptr ? 1 : 0, g_wait_ns.load(std::memory_order_relaxed),
+                                     take_stall(2));
     if (e != cudaSuccess) return cuda_fail("tile quantize launch", e);
     return last_launch_status("tile quantize launch");
 }
@@ -322,8 +325,29 @@ fp8_status fp8_quantize_act_1x128(const void* x_bf16, int64_t rows, int64_t cols
         return last_launch_status("row-wise quantize launch");
     }
     if (mode == FP8_COLWISE)
-        return launch_tile_quant<kTileColwise>(x_bf16, rows, cols, nullptr, nullptr, q_colT, s_col, s);
-    return launch_tile_quant<kTileBoth>(x_bf16, rows, cols, q_row, s_row, q_colT, s_col, s);
+        return launch_tile_quant<kTileColwise, false>(x_bf16, rows, cols, nullptr, nullptr, q_colT, s_col, s);
+    return launch_tile_quant<kTileBoth, false>(x_bf16, rows, cols, q_row, s_row, q_colT, s_col, s);
+}
+
+fp8_status fp8_swiglu_quantize_1x128(const void* gate_up_bf16, int64_t rows, int64_t ffn, int mode,
+                                     uint8_t* q_row, float* s_row, uint8_t* q_colT, float* s_col,
+                                     void* stream) {
+    if (mode != FP8_ROWWISE && mode != FP8_COLWISE && mode != FP8_BOTH) return FP8_ERR_MODE;
+    if (rows < 0 || ffn < 0 || rows % 128 || ffn % 128 || rows > kMaxDim || ffn > kMaxDim / 2)
+        return FP8_ERR_SHAPE;
+    if (rows == 0 || ffn == 0) return FP8_OK;
+    if (!gate_up_bf16) return FP8_ERR_NULL;
+    if ((mode & FP8_ROWWISE) && (!q_row || !s_row)) return FP8_ERR_NULL;
+    if ((mode & FP8_COLWISE) && (!q_colT || !s_col)) return FP8_ERR_NULL;
+    if (!aligned16(gate_up_bf16)) return FP8_ERR_ALIGN;
+    if ((mode & FP8_ROWWISE) && (!aligned16(q_row) || !aligned16(s_row))) return FP8_ERR_ALIGN;
+    if ((mode & FP8_COLWISE) && (!aligned16(q_colT) || !aligned16(s_col))) return FP8_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (mode == FP8_ROWWISE)
+        return launch_tile_quant<kTileRowwise, true>(gate_up_bf16, rows, ffn, q_row, s_row, nullptr, nullptr, s);
+    if (mode == FP8_COLWISE)
+        return launch_tile_quant<kTileColwise, true>(gate_up_bf16, rows, ffn, nullptr, nullptr, q_colT, s_col, s);
+    return launch_tile_quant<kTileBoth, true>(gate_up_bf16, rows, ffn, q_row, s_row, q_colT, s_col, s);
 }
 
 fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k, uint8_t* wq,
@@ -333,7 +357,7 @@ fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k,
     if (!w_bf16 || !wq || !sw) return FP8_ERR_NULL;
     if (!aligned16(w_bf16) || !aligned16(wq) || !aligned16(sw) || (wqT && !aligned16(wqT)))
         return FP8_ERR_ALIGN;
-    return launch_tile_quant<kTileWeight>(w_bf16, n, k, wq, nullptr, wqT, sw,
+    return launch_tile_quant<kTileWeight, false>(w_bf16, n, k, wq, nullptr, wqT, sw,
                                           static_cast<cudaStream_t>(stream));
 }
 
@@ -453,6 +477,13 @@ fp8_status fp8_selftest_division(unsigned long long* result, void* stream) {
     if (!aligned16(result)) return FP8_ERR_ALIGN;
     division_selftest_kernel<<<0x7F7F, 256, 0, static_cast<cudaStream_t>(stream)>>>(result);
     return last_launch_status("division self-test launch");
+}
+
+fp8_status fp8_selftest_silu_bf16(uint16_t* out, void* stream) {
+    if (!out) return FP8_ERR_NULL;
+    if (!aligned16(out)) return FP8_ERR_ALIGN;
+    silu_selftest_kernel<<<256, 256, 0, static_cast<cudaStream_t>(stream)>>>(out);
+    return last_launch_status("silu self-test launch");
 }
 
 fp8_status fp8_selftest_stall_next(int which) {

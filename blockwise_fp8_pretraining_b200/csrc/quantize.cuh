@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "swiglu.cuh"
 
 namespace fp8blk {
 
@@ -173,23 +174,32 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(const uint4* __restr
 
 // ---------------------------------------------------------------- 128x128 tiles
 
-enum TileMode : int { kTileColwise = 0, kTileBoth = 1, kTileWeight = 2 };
+// kTileRowwise is used with the SwiGLU input stage only; plain row-wise
+// groups have the lighter quant_rowwise_kernel.
+enum TileMode : int { kTileColwise = 0, kTileBoth = 1, kTileWeight = 2, kTileRowwise = 3 };
 
 namespace tile {
 constexpr int THREADS = 256;
 constexpr int BOX_BYTES = kGroup * 128;              // 128 rows x 64 bf16, 128-byte swizzle
-constexpr int IN_BYTES = 2 * BOX_BYTES;              // one bf16 tile = two boxes
 constexpr int OUT_BYTES = kGroup * kGroup;           // one tile of codes
-constexpr int OFF_IN0 = 0;
-constexpr int OFF_IN1 = OFF_IN0 + IN_BYTES;
-constexpr int OFF_ROW = OFF_IN1 + IN_BYTES;          // row-layout codes, 128-byte swizzle
-constexpr int OFF_COL = OFF_ROW + OUT_BYTES;         // transposed codes, 128-byte swizzle
-constexpr int OFF_RED = OFF_COL + OUT_BYTES;         // 4 x 128 floats of partial maxima
-constexpr int OFF_COLS = OFF_RED + 4 * kGroup * 4;   // 128 column scales, then their reciprocals
-constexpr int OFF_BARS = OFF_COLS + 2 * kGroup * 4;
-constexpr int SMEM_BYTES = OFF_BARS + 2 * 8 + 16 + 1024;   // + alignment slack
-static_assert(OFF_ROW % 1024 == 0 && OFF_COL % 1024 == 0 && BOX_BYTES % 1024 == 0,
-              "swizzled tiles must be 1024-byte aligned");
+// Shared-memory layout.  SWIGLU: a tile buffer holds the gate tile (two
+// boxes) and then the up tile (two boxes); h is written over the gate tile.
+template <bool SWIGLU>
+struct Layout {
+    static constexpr int IN_BYTES = (SWIGLU ? 4 : 2) * BOX_BYTES;
+    static constexpr int OFF_IN0 = 0;
+    static constexpr int OFF_IN1 = OFF_IN0 + IN_BYTES;
+    static constexpr int OFF_ROW = OFF_IN1 + IN_BYTES;          // row-layout codes, 128-byte swizzle
+    static constexpr int OFF_COL = OFF_ROW + OUT_BYTES;         // transposed codes, 128-byte swizzle
+    static constexpr int OFF_RED = OFF_COL + OUT_BYTES;         // 4 x 128 floats of partial maxima
+    static constexpr int OFF_COLS = OFF_RED + 4 * kGroup * 4;   // 128 column scales, then reciprocals
+    static constexpr int OFF_BARS = OFF_COLS + 2 * kGroup * 4;
+    static constexpr int SMEM_BYTES = OFF_BARS + 2 * 8 + 16 + 1024;   // + alignment slack
+    static constexpr int BLOCKS_PER_SM = SWIGLU ? 1 : 2;
+    static_assert(OFF_ROW % 1024 == 0 && OFF_COL % 1024 == 0 && BOX_BYTES % 1024 == 0,
+                  "swizzled tiles must be 1024-byte aligned");
+    static_assert(BLOCKS_PER_SM * SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
 
 // Byte offset of 16-byte chunk `chunk` of row `r` in a 128-byte-swizzled
 // tile of 128-byte rows (the TMA 128B swizzle pattern).
@@ -205,23 +215,30 @@ __device__ __forceinline__ int sw128(int r, int chunk) { return r * 128 + ((chun
 //   kTileWeight  : 128 x 128 blocks: q_row = codes [rows, cols], s_col =
 //                  block scales [rows/128, cols/128], transposed codes
 //                  through tmQT when has_qT
-// Maps (all 128-byte swizzle): tmX bf16 [rows, cols], box 64 x 128;
-//   tmQ u8 [rows, cols], box 128 x 128; tmQT u8 [cols, rows], box 128 x 128.
+//   kTileRowwise : groups along rows only (SWIGLU only)
+// SWIGLU: the quantized tensor is h = bf16(bf16(silu(gate)) * up) of a
+// gate_up activation [rows, 2 * cols] (gate = columns [0, cols), up =
+// [cols, 2 * cols)); each tile buffer receives the gate and the up tile of
+// the same position, and h is formed in place before the passes.
+// Maps (all 128-byte swizzle): tmX bf16 [rows, cols] (SWIGLU: [rows,
+//   2 * cols]), box 64 x 128; tmQ u8 [rows, cols], box 128 x 128; tmQT u8
+//   [cols, rows], box 128 x 128.
 // Row pass: lanes l and l + 16 of warp w share row 16 w + l % 16, 64 columns each.
 // Column pass: thread owns columns 2p, 2p+1 over the 32 rows of quarter qq.
-template <int MODE>
-__global__ void __launch_bounds__(tile::THREADS, 2)
+template <int MODE, bool SWIGLU>
+__global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PER_SM)
     quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmQT, int64_t rows, int64_t cols,
                       float* __restrict__ s_row, float* __restrict__ s_col, int has_qT,
                       uint64_t wait_ns, uint32_t stall_tx) {
+    using L = tile::Layout<SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
-    float* red = reinterpret_cast<float*>(smem + tile::OFF_RED);
-    const uint32_t bar0 = sbase + tile::OFF_BARS;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + tile::OFF_BARS + 16);
+    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
+    const uint32_t bar0 = sbase + L::OFF_BARS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_BARS + 16);
 
     const int t = threadIdx.x;
     const int lane = t & 31;
@@ -229,17 +246,22 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
     const int64_t tiles_c = cols / kGroup;
     const int64_t total = (rows / kGroup) * tiles_c;
     const bool want_rows = (MODE != kTileColwise);
-    const bool want_cols = (MODE != kTileWeight) || has_qT;
+    const bool want_cols = (MODE == kTileColwise || MODE == kTileBoth) || (MODE == kTileWeight && has_qT);
 
     // stall_tx (test only, 0 normally): extra bytes the block's first load
     // barrier expects, so that its wait runs out
     auto issue_load = [&](int64_t tl, int j) {
-        const uint32_t dst = sbase + (j ? tile::OFF_IN1 : tile::OFF_IN0);
+        const uint32_t dst = sbase + (j ? L::OFF_IN1 : L::OFF_IN0);
         const int32_t x = static_cast<int32_t>((tl % tiles_c) * kGroup);
         const int32_t y = static_cast<int32_t>((tl / tiles_c) * kGroup);
-        mbar_arrive_expect_tx(bar0 + 8 * j, tile::IN_BYTES + (tl == blockIdx.x ? stall_tx : 0u));
+        mbar_arrive_expect_tx(bar0 + 8 * j, L::IN_BYTES + (tl == blockIdx.x ? stall_tx : 0u));
         tma_load_2d(dst, &tmX, x, y, bar0 + 8 * j);
         tma_load_2d(dst + tile::BOX_BYTES, &tmX, x + 64, y, bar0 + 8 * j);
+        if (SWIGLU) {                  // the up tile, cols columns to the right
+            const int32_t xu = x + static_cast<int32_t>(cols);
+            tma_load_2d(dst + 2 * tile::BOX_BYTES, &tmX, xu, y, bar0 + 8 * j);
+            tma_load_2d(dst + 3 * tile::BOX_BYTES, &tmX, xu + 64, y, bar0 + 8 * j);
+        }
     };
 
     griddep_wait();                    // inputs of the preceding kernel are complete
@@ -278,10 +300,22 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
         const int b = i & 1;
         const int64_t tr = tl / tiles_c, tc = tl - tr * tiles_c;
         const int64_t r0 = tr * kGroup, c0 = tc * kGroup;
-        const uint8_t* tin = smem + (b ? tile::OFF_IN1 : tile::OFF_IN0);
+        const uint8_t* tin = smem + (b ? L::OFF_IN1 : L::OFF_IN0);
         bool ok = mbar_wait(bar0 + 8 * b, (i >> 1) & 1, abort_flag, wait_ns, kErrTimeout);
         if (t == 0) bulk_wait_group_read0();         // previous tile's stores have read the staging
         if (__syncthreads_or(!ok)) break;
+
+        if (SWIGLU) {
+            // ---- h over the gate tile (same swizzled layout as the up tile)
+            uint8_t* gbuf = smem + (b ? L::OFF_IN1 : L::OFF_IN0);
+#pragma unroll 2
+            for (int c = t; c < 2 * tile::BOX_BYTES / 16; c += tile::THREADS) {
+                const uint4 g = *reinterpret_cast<const uint4*>(gbuf + 16 * c);
+                const uint4 u = *reinterpret_cast<const uint4*>(gbuf + 2 * tile::BOX_BYTES + 16 * c);
+                *reinterpret_cast<uint4*>(gbuf + 16 * c) = swiglu8(g, u);
+            }
+            __syncthreads();
+        }
 
         // ---- row pass
         const uint8_t* myrow = tin + rbox * tile::BOX_BYTES;
@@ -311,7 +345,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
         if (want_rows) {
             const float sc = (MODE == kTileWeight) ? block_scale : group_scale(a);
             if (MODE != kTileWeight && rbox == 0) s_row[tc * rows + r0 + rrow] = sc;
-            uint8_t* orow = smem + tile::OFF_ROW;
+            uint8_t* orow = smem + L::OFF_ROW;
             const Quotient q(sc);
             uint32_t out[16];
             if (q.fast) {
@@ -355,7 +389,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
                 red[qq * kGroup + 2 * p + 1] = __uint_as_float(mu & 0xFFFF0000u);
                 __syncthreads();
                 // one thread per column finishes its scale and reciprocal
-                float* col_s = reinterpret_cast<float*>(smem + tile::OFF_COLS);
+                float* col_s = reinterpret_cast<float*>(smem + L::OFF_COLS);
                 if (t < kGroup) {
                     const float am = fmaxf(fmaxf(red[t], red[kGroup + t]),
                                            fmaxf(red[2 * kGroup + t], red[3 * kGroup + t]));
@@ -377,7 +411,7 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
             const Quotient q0(s0, rc0), q1(s1, rc1);
             const bool fast = q0.fast && q1.fast;
             const QuotientPair qp(s0, rc0, s1, rc1);
-            uint8_t* ocol = smem + tile::OFF_COL;
+            uint8_t* ocol = smem + L::OFF_COL;
             // Codes of rows 4j .. 4j+3 of 16-token chunk 2qq + h for both
             // columns, gathered into one word per column (row 4j lowest).
             auto gather16 = [&](auto&& code_of, int h, uint32_t (&b0)[4], uint32_t (&b1)[4]) {
@@ -417,9 +451,9 @@ __global__ void __launch_bounds__(tile::THREADS, 2)
         __syncthreads();
         if (t == 0) {
             if (want_rows)
-                tma_store_2d(&tmQ, sbase + tile::OFF_ROW, static_cast<int32_t>(c0), static_cast<int32_t>(r0));
+                tma_store_2d(&tmQ, sbase + L::OFF_ROW, static_cast<int32_t>(c0), static_cast<int32_t>(r0));
             if (want_cols)
-                tma_store_2d(&tmQT, sbase + tile::OFF_COL, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
+                tma_store_2d(&tmQT, sbase + L::OFF_COL, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
             bulk_commit_group();
             const int64_t nxt = tl + 2 * static_cast<int64_t>(gridDim.x);
             if (nxt < total) issue_load(nxt, b);

@@ -110,6 +110,28 @@ fp8_status fp8_quantize_act_1x128(const void *x_bf16, int64_t rows, int64_t cols
                                   uint8_t *q_colT, float *s_col, void *stream);
 
 /*
+ * Fused SwiGLU producer: h = bf16(bf16(silu(g)) * u) of a gate_up
+ * activation, quantized like fp8_quantize_act_1x128 quantizes a bf16 H,
+ * without writing H to memory.  g = gate_up[r, j] and u = gate_up[r, ffn + j]
+ * for j < ffn (the gate rows of the fused gate_up weight come first).  silu
+ * is rounded once, correctly, to bfloat16, then the product; the codes and
+ * scales equal those of fp8_quantize_act_1x128 on that H bit for bit.
+ * Passage: Puro-2B-Base model card (friendli.ai): model property table
+ * (Qwen3-1.7B configuration, gated SiLU feed-forward of size 6144) and
+ * training-setup paragraph (blockwise E4M3 linear-layer GEMMs, other
+ * activations in BF16).
+ *
+ *   gate_up_bf16 [rows, 2 * ffn] bf16, 16-byte aligned.
+ *   rows >= 0 and ffn >= 0, multiples of 128.
+ *   mode, q_row, s_row, q_colT, s_col: as fp8_quantize_act_1x128 with
+ *   cols = ffn (H is [rows, ffn]).
+ * rows == 0 or ffn == 0 is a no-op (pointers may then be NULL).
+ */
+fp8_status fp8_swiglu_quantize_1x128(const void *gate_up_bf16, int64_t rows, int64_t ffn,
+                                     int mode, uint8_t *q_row, float *s_row,
+                                     uint8_t *q_colT, float *s_col, void *stream);
+
+/*
  * Weight quantizer, 128x128 blocks.
  * Passage: Puro-2B-Base model card, training-setup paragraph (blockwise E4M3);
  * the 128x128 block follows the DeepSeek-V3 recipe the Puro-2B tech report
@@ -245,6 +267,12 @@ fp8_status fp8_selftest_division(unsigned long long *result, void *stream);
  * records FP8_ERR_TIMEOUT in the sticky error word.  For testing the timeout
  * path; nothing else is touched. */
 fp8_status fp8_selftest_wait_timeout(void *stream);
+
+/* out[b] = the bfloat16 bits of silu(g) as fp8_swiglu_quantize_1x128
+ * computes it, for the bfloat16 g with bits b, every b in 0..65535 (for
+ * checking it exhaustively).  out: 65536 device uint16, 16-byte aligned.
+ * Non-finite g are outside the definition. */
+fp8_status fp8_selftest_silu_bf16(uint16_t *out, void *stream);
 
 /* Arms the next launch of a kernel family so that the first operand
  * barrier of every CTA (pair) expects 16 bytes more than its copies bring:

@@ -173,3 +173,15 @@ def test_wgrad_accum_rejections(lib):
     assert g(P(A16), P(A16), P(A16), P(A16), P(A16), 128, 100, 128, S) == SHAPE
     assert g(P(A16), P(A16), P(A16), P(A16), None, 128, 128, 128, S) == NULL
     assert g(P(A16), P(A16), P(A16), P(A16), P(MIS), 128, 128, 128, S) == ALIGN
+
+
+def test_swiglu_quantize_rejections(lib):
+    q = lib.fp8_swiglu_quantize_1x128
+    assert q(P(A16), 256, 128, 0, P(A16), P(A16), None, None, S) == MODE
+    assert q(P(A16), 100, 128, 1, P(A16), P(A16), None, None, S) == SHAPE      # rows % 128
+    assert q(P(A16), 256, 100, 1, P(A16), P(A16), None, None, S) == SHAPE
+    assert q(None, 256, 128, 1, P(A16), P(A16), None, None, S) == NULL
+    assert q(P(A16), 256, 128, 2, None, None, P(A16), None, S) == NULL
+    assert q(P(MIS), 256, 128, 1, P(A16), P(A16), None, None, S) == ALIGN
+    assert q(P(A16), 0, 128, 3, None, None, None, None, S) == OK
+    assert lib.fp8_selftest_silu_bf16(None, S) == NULL

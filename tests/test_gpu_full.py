@@ -29,7 +29,7 @@ import blockwise_fp8_pretraining_b200 as fp8
 import oracle
 from blockwise_fp8_pretraining_b200 import synthetic as syn
 
-from _parity import (assert_within_bound, check_act, check_dgrad, check_fprop, check_wgrad,
+from _parity import (assert_bits_equal, assert_within_bound, check_act, check_dgrad, check_fprop, check_wgrad,
                      check_weight, dev, pick_rows)
 
 pytestmark = pytest.mark.gpu
@@ -84,8 +84,24 @@ def test_swiglu_mlp_fprop():
     gu, gu_bound = oracle.gemm_fprop(xq_o, sx_o, wq_o, sw_o)
     assert_within_bound(gu_gpu, gu, gu_bound, "gate_up fprop")
     del gu_gpu, gu_bound, xq, sx, wq, sw
-    h = syn.swiglu_bf16(torch.from_numpy(gu).to(torch.bfloat16))
+    gu_b = torch.from_numpy(gu).to(torch.bfloat16)
     del gu
+    # the fused SwiGLU producer on the bf16 gate_up output: H's codes and
+    # scales in both layouts, bit for bit against the oracle's SwiGLU
+    # followed by its quantizers
+    q_row, s_row, q_colT, s_col = fp8.fp8_swiglu_quantize_1x128(gu_b.to(d), fp8.BOTH)
+    torch.cuda.synchronize()
+    h_o = oracle.swiglu_bf16(syn.bf16_bits(gu_b))
+    q_o, s_o = oracle.quantize_act_rowwise(h_o)
+    assert_bits_equal(q_row, q_o, "fused H row-wise codes")
+    assert_bits_equal(s_row, s_o, "fused H row-wise scales")
+    q_o, s_o = oracle.quantize_act_colwise(h_o)
+    assert_bits_equal(q_colT, q_o, "fused H column-wise codes")
+    assert_bits_equal(s_col, s_o, "fused H column-wise scales")
+    del q_row, s_row, q_colT, s_col, h_o, q_o, s_o
+    # the unfused path: H from bf16 torch ops, as the configuration states
+    h = syn.swiglu_bf16(gu_b)
+    del gu_b
     check_act(h, fp8.BOTH)
     check_fprop(h, w_down, None, "down fprop")
 

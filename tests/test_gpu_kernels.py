@@ -377,6 +377,57 @@ def test_gemm_and_quantizer_time_out_drain_and_recover():
     finally:
         fp8.fp8_set_wait_timeout_ns(0)
         fp8.fp8_clear_error()
-    check_fprop(x, w)
+    check_fprop(x, w, output_rounding=True)
     check_act(x, fp8.COLWISE)
     assert fp8.fp8_get_error() == 0
+
+
+# ------------------------------------------------------ fused SwiGLU producer
+
+def test_silu_matches_the_oracle_on_every_finite_bfloat16():
+    """The fused producer's silu, rounded once to bfloat16, for all 65,024
+    finite bfloat16 inputs against the oracle's correctly rounded silu."""
+    got = fp8.fp8_selftest_silu_bf16()
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = ((bits.astype(np.uint32) >> 7) & 0xFF) != 0xFF
+    want = oracle.silu_bf16(bits[finite])
+    bad = np.nonzero(got[finite] != want)[0]
+    assert bad.size == 0, (f"{bad.size} inputs differ, first g=0x{int(bits[finite][bad[0]]):04x}: "
+                           f"gpu 0x{int(got[finite][bad[0]]):04x} oracle 0x{int(want[bad[0]]):04x}")
+
+
+def _gate_up_case(rows, ffn, seed):
+    """gate_up [rows, 2 ffn] bf16: N(0, 2) gate and N(0, 1) up, plus every
+    kind of special value silu and the product meet: zeros of both signs,
+    bfloat16 subnormals, values whose silu underflows FP32's exp, large
+    magnitudes, and products below FP32's normal range."""
+    g = syn.generator(seed)
+    gate = torch.randn((rows, ffn), generator=g) * 2.0
+    up = torch.randn((rows, ffn), generator=g)
+    special = torch.tensor([0.0, -0.0, 1e-40, -1e-40, 3e-39, -9.2e-41, 2.0 ** -31, -(2.0 ** -25),
+                            -90.0, -95.5, -100.0, -88.7, 85.0, -250.0, 300.0, 1e30, -1e30,
+                            2.0 ** -8, -(2.0 ** -8), 0.5, -0.5, 7.0, -7.0, 80.0, -80.0])
+    n = special.numel()
+    gate[0, :n] = special
+    gate[1, :n] = special
+    up[1, :n] = torch.tensor([1e-30] * n)            # products below 2^-126
+    gate[2, :n] = torch.full((n,), 1e-20)
+    up[2, :n] = special                               # tiny silu times everything
+    return torch.cat([gate, up], dim=1).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("rows,ffn", [(128, 128), (256, 384), (384, 2048)])
+@pytest.mark.parametrize("mode", [fp8.ROWWISE, fp8.COLWISE, fp8.BOTH])
+def test_swiglu_quantize_matches_the_unfused_definition(rows, ffn, mode):
+    gu = _gate_up_case(rows, ffn, rows + ffn + mode)
+    q_row, s_row, q_colT, s_col = fp8.fp8_swiglu_quantize_1x128(gu.to(dev()), mode)
+    torch.cuda.synchronize()
+    h = oracle.swiglu_bf16(syn.bf16_bits(gu))
+    if mode & fp8.ROWWISE:
+        q_o, s_o = oracle.quantize_act_rowwise(h)
+        assert_bits_equal(q_row, q_o, "fused row-wise codes")
+        assert_bits_equal(s_row, s_o, "fused row-wise scales")
+    if mode & fp8.COLWISE:
+        q_o, s_o = oracle.quantize_act_colwise(h)
+        assert_bits_equal(q_colT, q_o, "fused column-wise codes")
+        assert_bits_equal(s_col, s_o, "fused column-wise scales")
