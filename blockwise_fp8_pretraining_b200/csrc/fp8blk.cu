@@ -248,8 +248,11 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Para
 
     CUtensorMap ma, mb, mc;
     if ((st = make_operand_map(&ma, a, p.M, p.K, gemm::BM)) != FP8_OK) return st;
-    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::B_ROWS)) != FP8_OK) return st;
+    if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN / 2)) != FP8_OK) return st;
+    // (main-gradient mode writes through p.out_f32; the map still needs a
+    // valid encoding)
     if ((st = make_output_map(&mc, out, p.M, p.N, OUT == gemm::kOutAccF32)) != FP8_OK) return st;
+    if (OUT == gemm::kOutAccF32) p.out_f32 = static_cast<float*>(out);
 
     p.tiles_m = static_cast<int>((p.M + 2 * gemm::BM - 1) / (2 * gemm::BM));
     p.tiles_n = static_cast<int>((p.N + gemm::BN - 1) / gemm::BN);
@@ -281,7 +284,7 @@ bool dims_ok_gemm(int64_t M, int64_t N, int64_t K, bool m_positive) {
     if (m_positive && M == 0) return false;
     if (M % 128 || N % 128 || K % 128) return false;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return false;
-    if (static_cast<int64_t>((M + 255) / 256) * ((N + 191) / 192) > kMaxDim) return false;
+    if (static_cast<int64_t>((M + 255) / 256) * ((N + gemm::BN - 1) / gemm::BN) > kMaxDim) return false;
     return true;
 }
 

@@ -8,12 +8,14 @@
 // (part 7/7, section 5) cites: every slab's partial sum leaves the tensor
 // core in FP32 and is scaled before it joins the running FP32 accumulator.
 // The result is either rounded to BF16 and stored, or (main-gradient mode)
-// added in FP32 to the FP32 array already in memory.
+// added in FP32 to the FP32 array already in memory (vector reductions
+// straight from the registers, round-to-nearest-even; a subnormal sum may
+// be flushed to zero).
 //
-// Structure: clusters of two CTAs (one per SM) compute 256 x 192 output
-// tiles; persistent, 512 threads (4 warpgroups) per CTA.
+// Structure: clusters of two CTAs (one per SM) compute 256 x 256 output
+// tiles; persistent, 384 threads (3 warpgroups) per CTA.
 //   warp 0      operand producer (both CTAs): TMA loads of this CTA's 128
-//               rows of A and 96 rows of B per slab into a ring of
+//               rows of A and 128 rows of B per slab into a 4-deep ring of
 //               128-byte-swizzled stages, counted on the leader CTA's
 //               barrier (plain loads; no multicast anywhere).
 //   warp 2      scale producer (both CTAs): the scale vectors of 8 slabs at
@@ -23,24 +25,28 @@
 //               wait and one arrive per 8 slabs).  Both producers sleep
 //               between polls.
 //   warps 1, 3  MMA issuers (leader CTA only), warp 1 for even slabs and warp
-//               3 for odd slabs: 4 x tcgen05.mma.cta_group::2 (M=256, N=192,
-//               K=32, E4M3 -> F32) per slab into the slab's TMEM buffer (two,
-//               alternating, 256 columns apart), fresh every slab; each CTA's
-//               TMEM receives its 128 rows.  Commits free both CTAs' smem
-//               stage and publish the TMEM buffer to both CTAs' promotion
-//               warps.
-//   warps 4..15 promotion + epilogue (both CTAs, three warpgroups): each
-//               thread owns one output row (its TMEM lane) and 64 columns.
-//               Per slab it loads all 64 partials with two tcgen05.ld,
-//               hands the buffer back to the leader as soon as they have
-//               landed, and only then does acc = fma(c, P, acc) with packed
-//               FP32x2 FMAs, so the buffer is held for the load latency
-//               alone and the promotion of slab t overlaps the MMAs of slabs
-//               t+1 and t+2.  After the last slab it writes the tile through
-//               a per-warp 128-byte-swizzled staging buffer and a TMA store
-//               (BF16) or TMA reduce-add (FP32).
-// A thread's 64 columns start at a multiple of 64, so they never straddle a
-// 128-column weight block.
+//               3 for odd slabs: 4 x tcgen05.mma.cta_group::2 (M=256, N=256,
+//               K=32, E4M3 -> F32) per slab into the slab's 256-column TMEM
+//               buffer (two, alternating), fresh every slab; each CTA's TMEM
+//               receives its 128 rows.  Commits free both CTAs' smem stage
+//               and publish the TMEM buffer to both CTAs' promotion warps.
+//   warps 4..11 promotion + epilogue (both CTAs): each thread owns one output
+//               row (TMEM lane) and 128 columns.  Per slab it loads the
+//               partials with tcgen05.ld into two 32-column register sets
+//               (the next chunk is loaded into a set as soon as its FMAs have
+//               read it), hands the TMEM buffer back to the leader once the
+//               last chunk has landed, and does acc = fma(c, P, acc) in
+//               registers with packed FP32x2 FMAs.  After the last slab it
+//               writes the tile through a per-warp 128-byte-swizzled staging
+//               buffer and a TMA store (BF16), or adds it to the FP32 array
+//               with vector reductions.
+// Why this shape: the MMA of slab t+2 reuses the buffer of slab t, so each
+// slab's hand-off (commit -> wake -> loads -> release -> issue, about 1 us
+// measured on B200) must fit in the time of two slabs' MMAs.  A 256-column
+// tile gives the most MMA work per hand-off that two buffers of tensor
+// memory can hold; narrower tiles with more buffers, or a whole slab staged
+// in registers by more promotion warps, measured slower (the operand feed of
+// narrower tiles is slower, and more waiters per barrier wake later).
 // Scale modes:
 //   kScaleRowBlock (fprop, dgrad): s_a is per output row (1x128 activation
 //     groups), s_b per 128-column block of the weight (128x128 blocks), so
@@ -63,34 +69,34 @@ namespace fp8blk {
 namespace gemm {
 
 constexpr int BM = 128;              // output rows per CTA (256 per pair)
-constexpr int BN = 192;              // output columns per pair tile
+constexpr int BN = 256;              // output columns per pair tile
 constexpr int BK = 128;              // one quantization slab
 constexpr int UMMA_K = 32;           // K of one kind::f8f6f4 MMA
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int SCHUNK = 8;            // slabs of scales per ring slot
 constexpr int SSLOTS = 2;            // scale ring slots
 constexpr int A_BYTES = BM * BK;             // this CTA's 128 rows of A
-constexpr int B_ROWS = BN / 2;               // this CTA's 96 rows of B
-constexpr int B_BYTES = B_ROWS * BK;
+constexpr int B_BYTES = (BN / 2) * BK;       // this CTA's 128 rows of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;
-constexpr int COLS_PER_WARP = 64;            // output columns per promotion thread
-constexpr int EPI_WARPS = 4 * (BN / COLS_PER_WARP);   // 12
-constexpr int EPI_WARP0 = 4;         // first promotion warp (warpgroups 1..3)
-constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;  // 512
-// Register split: launched at 128 per thread (512 x 128 = 65536).  Warpgroup
-// 0 drops to 56 and the three promotion warpgroups rise to 152
-// (128 x 56 + 384 x 152 = 65536): 64 accumulators, 64 staged partials.
-constexpr int REGS_LAUNCH = 128;
-constexpr int REGS_PRODUCER = 56;
-constexpr int REGS_EPILOGUE = 152;
-static_assert(128 * REGS_PRODUCER + 384 * REGS_EPILOGUE <= THREADS * REGS_LAUNCH,
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARP0 = 4;         // first epilogue warp (warpgroups 1 and 2)
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
+// Register split: launched at 168 per thread (384 x 168 = 64512).  Row-block
+// mode: warpgroup 0 drops to 72 and the two epilogue warpgroups rise to 216
+// (128 x 72 + 256 x 216 = 64512); at 40 the producer roles spill.  Outer mode
+// needs more in the epilogue (the per-column scale products): 40 / 232.
+constexpr int REGS_LAUNCH = 168;
+template <int SCALE> struct RegSplit;
+template <> struct RegSplit<0> { static constexpr int producer = 72, epilogue = 216; };
+template <> struct RegSplit<1> { static constexpr int producer = 40, epilogue = 232; };
+static_assert(128 * RegSplit<0>::producer + 256 * RegSplit<0>::epilogue <= THREADS * REGS_LAUNCH,
               "register split exceeds the launch allocation");
-static_assert(THREADS * REGS_LAUNCH <= 65536, "launch allocation exceeds the register file");
-constexpr int TMEM_COLS = 512;
-constexpr int TMEM_BUF_STRIDE = 256;         // buffer b at column 256 b
+static_assert(128 * RegSplit<1>::producer + 256 * RegSplit<1>::epilogue <= THREADS * REGS_LAUNCH,
+              "register split exceeds the launch allocation");
+constexpr int TMEM_COLS = 2 * BN;
 constexpr int SCALE_SLOT_BYTES = SCHUNK * (BM + BN) * 4;   // s_a then s_b, slab-major
-constexpr int OUT_WARP_BYTES = 32 * 128;     // 32 rows x 128 bytes per promotion warp
+constexpr int OUT_WARP_BYTES = 32 * 128 * 2;     // 32 rows x 128 BF16 per epilogue warp
 
 constexpr int OFF_SCALES = STAGES * STAGE_BYTES;
 constexpr int OFF_OUT = OFF_SCALES + SSLOTS * SCALE_SLOT_BYTES;
@@ -100,9 +106,8 @@ constexpr int OFF_TMEM_SLOT = OFF_BARS + NUM_BARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr int SMEM_BYTES = OFF_ABORT + 4 + 1024;   // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(OFF_OUT % 1024 == 0 && OFF_SCALES % 1024 == 0, "1024-byte alignment of staging");
+static_assert(OFF_OUT % 1024 == 0, "swizzled staging must be 1024-byte aligned");
 static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzled stages must be 1024-byte aligned");
-static_assert(BN % 64 == 0 && BN <= TMEM_BUF_STRIDE, "tile width");
 
 constexpr uint32_t IDESC = idesc_e4m3_f32(2 * BM, BN);
 
@@ -114,6 +119,7 @@ enum OutMode : int { kOutBf16 = 0, kOutAccF32 = 1 };
 // producer a chunk of 8 slabs ahead.
 constexpr uint32_t kProducerSleepNs = 128;
 constexpr uint32_t kScaleSleepNs = 256;
+constexpr uint32_t kIssuerSleepNs = 0;
 
 struct Params {
     const float* sa;        // s_a(t, i) = sa[t * sa_ld + i]
@@ -122,9 +128,10 @@ struct Params {
     int64_t sb_sn, sb_sk;   // outer:     s_b(t, j)  = sb[t * sb_ld + j]
     int64_t sb_ld;
     int M, N, K;            // output rows, output columns, contraction
-    int tiles_m, tiles_n;   // pair tiles: 256-row by 192-column
+    int tiles_m, tiles_n;   // pair tiles: 256-row by 256-column
     uint64_t wait_ns;
     uint32_t stall_tx;      // test only: extra bytes the first stage's barrier expects (0 normally)
+    float* out_f32;         // main-gradient mode: the FP32 array [M, N] added to
 };
 
 struct Bars {
@@ -137,38 +144,9 @@ struct Bars {
     __device__ __forceinline__ uint32_t sempty_(int s) const { return sempty + 8 * s; }
 };
 
-// acc[c0 .. c0+31] += coefficient * P with packed FP32x2 FMAs.  Row-block
-// mode: one coefficient (cpair) per thread and slab.  Outer mode: the
-// partials of column j are first multiplied by that column's scale sbv[j]
-// (this thread's column scales in shared memory), then acc = fma(sa, ., acc),
-// so no coefficient vector is held in registers.
-template <int SCALE>
-__device__ __forceinline__ void promote32(float (&acc)[64], const uint32_t (&r)[32], int c0, float2 cpair,
-                                          float sa, const float* sbv) {
-#pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-        const int a = c0 + j;
-        float2 p01 = make_float2(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
-        float2 p23 = make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-        float2 c01 = cpair, c23 = cpair;
-        if (SCALE == kScaleOuter) {
-            const float4 b4 = *reinterpret_cast<const float4*>(sbv + a);
-            p01 = __fmul2_rn(make_float2(b4.x, b4.y), p01);
-            p23 = __fmul2_rn(make_float2(b4.z, b4.w), p23);
-            c01 = c23 = make_float2(sa, sa);
-        }
-        const float2 v01 = __ffma2_rn(c01, p01, make_float2(acc[a + 0], acc[a + 1]));
-        const float2 v23 = __ffma2_rn(c23, p23, make_float2(acc[a + 2], acc[a + 3]));
-        acc[a + 0] = v01.x;
-        acc[a + 1] = v01.y;
-        acc[a + 2] = v23.x;
-        acc[a + 3] = v23.y;
-    }
-}
-
-// tmA: A codes [M, K] (box 128 x 128), tmB: B codes [N, K] (box 128 x 96),
-// tmC: output [M, N], BF16 with box 64 x 32 (kOutBf16) or FP32 with box
-// 32 x 32 (kOutAccF32), both 128-byte swizzled.
+// tmA: A codes [M, K] (box 128 x 128), tmB: B codes [N, K] (box 128 x 128),
+// tmC: BF16 output [M, N], box 64 x 32, 128-byte swizzled (kOutBf16; in
+// main-gradient mode p.out_f32 is written instead).
 template <int SCALE, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -202,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars.tfull_(b), 1);
-            mbar_init(bars.tempty_(b), 2 * EPI_WARPS);   // leader: both CTAs' promotion warps
+            mbar_init(bars.tempty_(b), 2 * EPI_WARPS);   // leader: both CTAs' epilogue warps
         }
         for (int s = 0; s < SSLOTS; ++s) {
             mbar_init(bars.sfull_(s), 1);
@@ -229,7 +207,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     griddep_wait();                                      // inputs of the preceding kernel are complete
 
     if (warp < EPI_WARP0) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<SCALE>::producer));
       if (warp == 0) {
         // ---------------------------------------------------- operand producer
         if (lane == 0) {
@@ -249,7 +227,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t a_dst = sbase + s * STAGE_BYTES;
                     if (rank == 0) mbar_arrive_expect_tx(bars.full_(s), PAIR_STAGE_BYTES + (it == 0 ? p.stall_tx : 0u));
                     tma_load_2d_pair(a_dst, &tmA, kb * BK, m_own, full_leader + 8 * s);
-                    tma_load_2d_pair(a_dst + A_BYTES, &tmB, kb * BK, n0 + static_cast<int>(rank) * B_ROWS,
+                    tma_load_2d_pair(a_dst + A_BYTES, &tmB, kb * BK, n0 + static_cast<int>(rank) * (BN / 2),
                                      full_leader + 8 * s);
                     ++it;
                 }
@@ -267,9 +245,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------ scale producer
         // Lane 0 issues the bulk copies of s_a (and, in outer mode, s_b).  In
         // row-block mode lanes 0..15 also fetch the chunk's weight-block
-        // scales (the two blocks a 192-column tile touches; strided in dgrad,
-        // so not a bulk copy) and store them into the slot before lane 0
-        // arrives.
+        // scales (two blocks per 256-column tile; strided in dgrad, so not a
+        // bulk copy) and store them into the slot before lane 0 arrives.
         int ic = 0;    // scale chunks requested
         bool ok = true;
         for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
@@ -319,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 drain_wait(bars.sfull_(j % SSLOTS), (j / SSLOTS) & 1, p.wait_ns);
         }
         __syncwarp();
-      } else {
+      } else if (warp == 1 || warp == 3) {
         // -------------------------------------------------- MMA issuer (leader)
         if (lane == 0 && rank == 0) {
             const int sel = (warp == 1) ? 0 : 1;
@@ -329,7 +306,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     if ((it & 1) != sel) continue;
                     const int buf = it & 1;
-                    if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout)) {
+                    if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout,
+                                   kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -342,7 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t a_addr = sbase + s * STAGE_BYTES;
                     const uint64_t a_desc = smem_desc_k128_sw128(a_addr);
                     const uint64_t b_desc = smem_desc_k128_sw128(a_addr + A_BYTES);
-                    const uint32_t d_tmem = tmem_base + buf * TMEM_BUF_STRIDE;
+                    const uint32_t d_tmem = tmem_base + buf * BN;
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // +32 bytes along K inside the swizzled 128-byte row
@@ -360,26 +338,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_EPILOGUE));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<SCALE>::epilogue));
         // ----------------------------------------------- promotion + epilogue
         const int ew = warp - EPI_WARP0;
         const int quarter = warp & 3;          // TMEM lanes this warp may read
-        const int cb = ew >> 2;                // which 64 of the tile's 192 columns
+        const int half = ew >> 2;              // which 128 of the 256 columns
         const int row_in_tile = quarter * 32 + lane;
-        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + cb * COLS_PER_WARP;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
         const uint32_t tempty_leader = map_to_cta(bars.tempty, 0);
 
-        float acc[64];
+        float acc[128];
         int it = 0;
         int ic = 0;        // scale chunks consumed
         bool ok = true;
         for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
             const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
             const int n0 = (tile % p.tiles_n) * BN;
-            // weight block of this thread's columns, relative to the tile's first block
-            const int blk = (n0 + cb * COLS_PER_WARP) / 128 - n0 / 128;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 
             for (int kb = 0; kb < num_kb; ++kb, ++it) {
                 const int buf = it & 1;
@@ -394,20 +370,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                // the whole slab share: 64 partials in two loads, one wait
-                uint32_t ra[32], rb[32];
-                const uint32_t taddr = lane_base + buf * TMEM_BUF_STRIDE;
-                tmem_ld_32x32b_x32(taddr, ra);
-                tmem_ld_32x32b_x32(taddr + 32, rb);
                 const float* slot =
                     reinterpret_cast<const float*>(smem + OFF_SCALES + sl * SCALE_SLOT_BYTES);
                 const float sa = slot[j_in_chunk * BM + row_in_tile];
+                const uint32_t taddr = lane_base + buf * BN + half * 128;
                 float2 cpair = make_float2(0.0f, 0.0f);
                 if (SCALE == kScaleRowBlock) {
-                    const float c = sa * slot[SCHUNK * BM + 2 * j_in_chunk + blk];
+                    const float c = sa * slot[SCHUNK * BM + 2 * j_in_chunk + half];
                     cpair = make_float2(c, c);
                 }
-                const float* sbv = slot + SCHUNK * BM + j_in_chunk * BN + cb * COLS_PER_WARP;
+                const float* sbv = slot + SCHUNK * BM + j_in_chunk * BN + half * 128;
+                // Promote 32 columns held in r (columns c0 .. c0+31 of this half)
+                // with packed FP32x2 FMAs: acc = c * partial + acc, two
+                // columns per instruction.
+                auto promote = [&](const uint32_t (&r)[32], int c0) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const int a = c0 + j;
+                        float2 p01 = make_float2(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
+                        float2 p23 = make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                        float2 c01 = cpair, c23 = cpair;
+                        if (SCALE == kScaleOuter) {
+                            // column scales into the partials, then the row scale
+                            const float4 b4 = *reinterpret_cast<const float4*>(sbv + a);
+                            p01 = __fmul2_rn(make_float2(b4.x, b4.y), p01);
+                            p23 = __fmul2_rn(make_float2(b4.z, b4.w), p23);
+                            c01 = c23 = make_float2(sa, sa);
+                        }
+                        const float2 v01 = __ffma2_rn(c01, p01, make_float2(acc[a + 0], acc[a + 1]));
+                        const float2 v23 = __ffma2_rn(c23, p23, make_float2(acc[a + 2], acc[a + 3]));
+                        acc[a + 0] = v01.x;
+                        acc[a + 1] = v01.y;
+                        acc[a + 2] = v23.x;
+                        acc[a + 3] = v23.y;
+                    }
+                };
+                // Two 32-column register sets: chunks 0 and 1 land, chunk 2
+                // and 3 loads are issued into a set as soon as its FMAs have
+                // read it, and the buffer goes back to the MMA issuer once
+                // chunks 2 and 3 have landed (two waits per slab).
+                uint32_t ra[32], rb[32];
+                tmem_ld_32x32b_x32(taddr, ra);
+                tmem_ld_32x32b_x32(taddr + 32, rb);
+                tmem_ld_wait();
+                promote(ra, 0);
+                tmem_ld_32x32b_x32(taddr + 64, ra);
+                promote(rb, 32);
+                tmem_ld_32x32b_x32(taddr + 96, rb);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -417,8 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     else
                         mbar_arrive_remote(tempty_leader + 8 * buf);
                 }
-                promote32<SCALE>(acc, ra, 0, cpair, sa, sbv);
-                promote32<SCALE>(acc, rb, 32, cpair, sa, sbv);
+                promote(ra, 64);
+                promote(rb, 96);
                 if (j_in_chunk == SCHUNK - 1 || kb == num_kb - 1) {
                     // last slab of this scale chunk: the slot may be refilled
                     __syncwarp();
@@ -428,63 +437,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             if (!ok) break;
 
-            // Output through this warp's staging buffer (32 rows of 128 bytes,
-            // 16-byte chunk c of row r at position c ^ (r % 8)).
-            const int col0 = n0 + cb * COLS_PER_WARP;
-            if (col0 < p.N && m_own < p.M) {
+            // BF16 round-to-nearest-even into this warp's staging buffer (two
+            // 32 x 64 boxes, 128-byte rows, 16-byte chunk j of row r at
+            // position j ^ (r % 8)), then TMA stores of the two boxes.
+            const int col0 = n0 + half * 128;
+            if (OUT == kOutAccF32 && col0 < p.N && m_own < p.M) {
+                // FP32 added to the array in memory straight from the
+                // registers: one vector reduction per 4 columns, so each
+                // element receives exactly one addition per call
+                float* dst = p.out_f32 + static_cast<int64_t>(m_own + quarter * 32 + lane) * p.N + col0;
+#pragma unroll
+                for (int j = 0; j < 128; j += 4)
+                    red_add_v4_f32(dst + j, acc[j + 0], acc[j + 1], acc[j + 2], acc[j + 3]);
+            } else if (OUT == kOutBf16 && col0 < p.N && m_own < p.M) {
                 // The row's staging address and swizzle key come out of an
-                // opaque move, so that the compiler computes the chunk
+                // opaque move, so that the compiler computes the 16 chunk
                 // addresses here instead of keeping them live across the slab loop.
                 uint32_t row_addr, key;
                 asm volatile("mov.u32 %0, %1;" : "=r"(row_addr) : "r"(smem_u32(smem + OFF_OUT + ew * OUT_WARP_BYTES) + lane * 128));
                 asm volatile("mov.u32 %0, %1;" : "=r"(key) : "r"((lane & 7) << 4));
-                const uint32_t src = smem_u32(smem + OFF_OUT + ew * OUT_WARP_BYTES);
-                const int row0 = m_own + quarter * 32;
-                if (OUT == kOutBf16) {
-                    // BF16 round-to-nearest-even, one 64-column box
-                    if (lane == 0) bulk_wait_group_read0();     // previous tile's store has read the buffer
-                    __syncwarp();
+                if (lane == 0) bulk_wait_group_read0();     // previous tile's store has read the buffer
+                __syncwarp();
 #pragma unroll
-                    for (int j = 0; j < 64; j += 8) {
-                        uint4 o;
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-                        __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
-                        o.x = *reinterpret_cast<uint32_t*>(&h0);
-                        o.y = *reinterpret_cast<uint32_t*>(&h1);
-                        o.z = *reinterpret_cast<uint32_t*>(&h2);
-                        o.w = *reinterpret_cast<uint32_t*>(&h3);
-                        st_shared_v4(row_addr + ((static_cast<uint32_t>(j >> 3) << 4) ^ key), o);
-                    }
-                    fence_proxy_async_shared();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmC, src, col0, row0);
-                        bulk_commit_group();
-                    }
-                } else {
-                    // FP32 added to the array in memory by TMA reduce-add, two
-                    // 32-column boxes through the same staging buffer
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (lane == 0) bulk_wait_group_read0();
-                        __syncwarp();
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const uint4 o = make_uint4(__float_as_uint(acc[32 * h + j + 0]),
-                                                       __float_as_uint(acc[32 * h + j + 1]),
-                                                       __float_as_uint(acc[32 * h + j + 2]),
-                                                       __float_as_uint(acc[32 * h + j + 3]));
-                            st_shared_v4(row_addr + ((static_cast<uint32_t>(j >> 2) << 4) ^ key), o);
-                        }
-                        fence_proxy_async_shared();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_reduce_add_2d(&tmC, src, col0 + 32 * h, row0);
-                            bulk_commit_group();
-                        }
-                    }
+                for (int j = 0; j < 128; j += 8) {
+                    uint4 o;
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+                    __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+                    o.x = *reinterpret_cast<uint32_t*>(&h0);
+                    o.y = *reinterpret_cast<uint32_t*>(&h1);
+                    o.z = *reinterpret_cast<uint32_t*>(&h2);
+                    o.w = *reinterpret_cast<uint32_t*>(&h3);
+                    const int box = j >> 6;                 // which 64-column box
+                    const int chunk = (j & 63) >> 3;        // 16-byte chunk in the 128-byte row
+                    st_shared_v4(row_addr + box * 4096 + ((static_cast<uint32_t>(chunk) << 4) ^ key), o);
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    const uint32_t src = smem_u32(smem + OFF_OUT + ew * OUT_WARP_BYTES);
+                    tma_store_2d(&tmC, src, col0, m_own + quarter * 32);
+                    tma_store_2d(&tmC, src + 4096, col0 + 64, m_own + quarter * 32);
+                    bulk_commit_group();
                 }
             }
         }

@@ -182,20 +182,25 @@ namespace tile {
 constexpr int THREADS = 256;
 constexpr int BOX_BYTES = kGroup * 128;              // 128 rows x 64 bf16, 128-byte swizzle
 constexpr int OUT_BYTES = kGroup * kGroup;           // one tile of codes
-// Shared-memory layout.  SWIGLU: a tile buffer holds the gate tile (two
-// boxes) and then the up tile (two boxes); h is written over the gate tile.
+// Shared-memory layout.  Plain tiles: two tile buffers, separate staging of
+// the two code tiles, two blocks per SM.  SWIGLU: one buffer holding the
+// gate tile (two boxes) and then the up tile (two boxes); h is written over
+// the gate tile, and the up tile, dead once h is formed, stages the codes;
+// three blocks per SM overlap each other's loads.
 template <bool SWIGLU>
 struct Layout {
+    static constexpr int NBUF = SWIGLU ? 1 : 2;
     static constexpr int IN_BYTES = (SWIGLU ? 4 : 2) * BOX_BYTES;
     static constexpr int OFF_IN0 = 0;
-    static constexpr int OFF_IN1 = OFF_IN0 + IN_BYTES;
-    static constexpr int OFF_ROW = OFF_IN1 + IN_BYTES;          // row-layout codes, 128-byte swizzle
+    static constexpr int OFF_IN1 = OFF_IN0 + (NBUF - 1) * IN_BYTES;
+    static constexpr int OFF_ROW = SWIGLU ? 2 * BOX_BYTES : OFF_IN1 + IN_BYTES;   // row-layout codes
     static constexpr int OFF_COL = OFF_ROW + OUT_BYTES;         // transposed codes, 128-byte swizzle
-    static constexpr int OFF_RED = OFF_COL + OUT_BYTES;         // 4 x 128 floats of partial maxima
+    static constexpr int OFF_RED = SWIGLU ? IN_BYTES : OFF_COL + OUT_BYTES;   // 4 x 128 partial maxima
     static constexpr int OFF_COLS = OFF_RED + 4 * kGroup * 4;   // 128 column scales, then reciprocals
     static constexpr int OFF_BARS = OFF_COLS + 2 * kGroup * 4;
     static constexpr int SMEM_BYTES = OFF_BARS + 2 * 8 + 16 + 1024;   // + alignment slack
-    static constexpr int BLOCKS_PER_SM = SWIGLU ? 1 : 2;
+    static constexpr int BLOCKS_PER_SM = SWIGLU ? 3 : 2;
+    static_assert(OFF_COL + OUT_BYTES <= (SWIGLU ? IN_BYTES : OFF_RED), "staging inside its region");
     static_assert(OFF_ROW % 1024 == 0 && OFF_COL % 1024 == 0 && BOX_BYTES % 1024 == 0,
                   "swizzled tiles must be 1024-byte aligned");
     static_assert(BLOCKS_PER_SM * SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -271,7 +276,7 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tmX);
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < L::NBUF; ++j) {
             const int64_t tl = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
             if (tl < total) issue_load(tl, j);
         }
@@ -297,11 +302,11 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
 
     int i = 0;
     for (int64_t tl = blockIdx.x; tl < total; tl += gridDim.x, ++i) {
-        const int b = i & 1;
+        const int b = i % L::NBUF;
         const int64_t tr = tl / tiles_c, tc = tl - tr * tiles_c;
         const int64_t r0 = tr * kGroup, c0 = tc * kGroup;
         const uint8_t* tin = smem + (b ? L::OFF_IN1 : L::OFF_IN0);
-        bool ok = mbar_wait(bar0 + 8 * b, (i >> 1) & 1, abort_flag, wait_ns, kErrTimeout);
+        bool ok = mbar_wait(bar0 + 8 * b, (i / L::NBUF) & 1, abort_flag, wait_ns, kErrTimeout);
         if (t == 0) bulk_wait_group_read0();         // previous tile's stores have read the staging
         if (__syncthreads_or(!ok)) break;
 
@@ -446,7 +451,7 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
             }
         }
 
-        // ---- stores of both code tiles, then the load two tiles ahead
+        // ---- stores of both code tiles, then the load NBUF tiles ahead
         fence_proxy_async_shared();
         __syncthreads();
         if (t == 0) {
@@ -455,17 +460,21 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
             if (want_cols)
                 tma_store_2d(&tmQT, sbase + L::OFF_COL, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
             bulk_commit_group();
-            const int64_t nxt = tl + 2 * static_cast<int64_t>(gridDim.x);
-            if (nxt < total) issue_load(nxt, b);
+            const int64_t nxt = tl + L::NBUF * static_cast<int64_t>(gridDim.x);
+            if (nxt < total) {
+                if (SWIGLU) bulk_wait_group_read0();    // the codes are staged in the buffer's up half
+                issue_load(nxt, b);
+            }
         }
     }
     griddep_launch_dependents();
     if (t == 0) {
         if (*abort_flag) {
             // let loads already requested land before the block exits
-            for (int j = 0; j < 2; ++j) {
+            for (int j = 0; j < L::NBUF; ++j) {
                 const int64_t tl = blockIdx.x + static_cast<int64_t>(i + j) * gridDim.x;
-                if (tl < total) drain_wait(bar0 + 8 * ((i + j) & 1), ((i + j) >> 1) & 1, wait_ns);
+                if (tl < total)
+                    drain_wait(bar0 + 8 * ((i + j) % L::NBUF), ((i + j) / L::NBUF) & 1, wait_ns);
             }
         }
         bulk_wait_group0();
