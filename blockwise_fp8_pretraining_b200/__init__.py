@@ -18,11 +18,14 @@ from ._abi import (  # noqa: F401
     fp8_block_gemm_wgrad_accum_f32,
     fp8_cast_e4m3_scaled,
     fp8_clear_error,
+    fp8_gemm_workspace,
+    fp8_gemm_workspace_bytes,
     fp8_get_error,
     fp8_last_cuda_error,
     fp8_quantize_act_1x128,
     fp8_quantize_weight_128x128,
     fp8_selftest_division,
+    fp8_selftest_gemm_schedule,
     fp8_selftest_silu_bf16,
     fp8_selftest_stall_next,
     fp8_selftest_wait_timeout,

@@ -53,21 +53,24 @@ def load() -> ctypes.CDLL:
         raise OSError(f"{path} is missing: build it with python -m blockwise_fp8_pretraining_b200.build")
     lib = ctypes.CDLL(path)
     p, i64, i32, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int
+    sz = ctypes.c_size_t
     sig = {
         "fp8_quantize_act_1x128": [p, i64, i64, i32, p, p, p, p, p],
         "fp8_quantize_weight_128x128": [p, i64, i64, p, p, p, p],
         "fp8_swiglu_quantize_1x128": [p, i64, i64, i32, p, p, p, p, p],
         "fp8_selftest_silu_bf16": [p, p],
-        "fp8_block_gemm_fprop": [p, p, p, p, p, i64, i64, i64, p],
-        "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p],
-        "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p],
-        "fp8_block_gemm_wgrad_accum_f32": [p, p, p, p, p, i64, i64, i64, p],
+        "fp8_block_gemm_fprop": [p, p, p, p, p, i64, i64, i64, p, sz, p],
+        "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p, sz, p],
+        "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p, sz, p],
+        "fp8_block_gemm_wgrad_accum_f32": [p, p, p, p, p, i64, i64, i64, p, sz, p],
+        "fp8_gemm_workspace_bytes": [p],
         "fp8_get_error": [],
         "fp8_clear_error": [],
         "fp8_set_wait_timeout_ns": [ctypes.c_uint64],
         "fp8_cast_e4m3_scaled": [p, ctypes.c_float, p, i64, p],
         "fp8_selftest_wait_timeout": [p],
         "fp8_selftest_stall_next": [i32],
+        "fp8_selftest_gemm_schedule": [i64, i64, i64, i32, i32, p, i64, p],
         "fp8_selftest_division": [p, p],
     }
     for name, args in sig.items():
@@ -240,9 +243,36 @@ def fp8_quantize_weight_128x128(w, wq=None, sw=None, wqT=None, transposed=True, 
     return wq, sw, wqT
 
 
-def fp8_block_gemm_fprop(xq, sx, wq, sw, y=None, stream=None):
+def _workspace(ws):
+    """(pointer, bytes) of an optional GEMM workspace tensor (see
+    fp8_gemm_workspace_bytes): contiguous, on the current device, zeroed
+    before its first use."""
+    if ws is None:
+        return ctypes.c_void_p(0), 0
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+
+def fp8_gemm_workspace_bytes() -> int:
+    """Bytes of the GEMM workspace on the current device."""
+    n = ctypes.c_size_t(0)
+    _check(load().fp8_gemm_workspace_bytes(ctypes.byref(n)), "fp8_gemm_workspace_bytes")
+    return int(n.value)
+
+
+def fp8_gemm_workspace(device=None) -> torch.Tensor:
+    """A zeroed GEMM workspace for the current (or given) device, allocated
+    by torch.  One launch at a time may use it."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return torch.zeros(fp8_gemm_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+
+def fp8_block_gemm_fprop(xq, sx, wq, sw, y=None, stream=None, workspace=None):
     """Y[M, N] = X W^T (bf16) from X codes [M, K] / scales [K/128, M] and W
-    codes [N, K] / scales [N/128, K/128]."""
+    codes [N, K] / scales [N/128, K/128].  workspace: optional (see
+    fp8_gemm_workspace)."""
     lib = load()
     M, K = xq.shape
     N = wq.shape[0]
@@ -252,15 +282,16 @@ def fp8_block_gemm_fprop(xq, sx, wq, sw, y=None, stream=None):
     _want(sw, torch.float32, (N // 128, K // 128), "sw")
     allocated = y is None
     y = _out(y, torch.bfloat16, (M, N), xq.device, "y")
-    _launch_checks([("xq", xq), ("sx", sx), ("wq", wq), ("sw", sw), ("y", y)], stream)
+    _launch_checks([("xq", xq), ("sx", sx), ("wq", wq), ("sw", sw), ("y", y), ("workspace", workspace)],
+                   stream)
     _record(stream, [y] if allocated else [])
     _check(lib.fp8_block_gemm_fprop(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K,
-                                    _stream(stream)),
+                                    *_workspace(workspace), _stream(stream)),
            "fp8_block_gemm_fprop")
     return y
 
 
-def fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=None, stream=None):
+def fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=None, stream=None, workspace=None):
     """dX[M, K] = dY W (bf16) from dY codes [M, N] / scales [N/128, M], the
     transposed weight codes [K, N] and the weight scales [N/128, K/128]."""
     lib = load()
@@ -272,15 +303,16 @@ def fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=None, stream=None):
     _want(sw, torch.float32, (N // 128, K // 128), "sw")
     allocated = dx is None
     dx = _out(dx, torch.bfloat16, (M, K), dyq.device, "dx")
-    _launch_checks([("dyq", dyq), ("sdy", sdy), ("wqT", wqT), ("sw", sw), ("dx", dx)], stream)
+    _launch_checks([("dyq", dyq), ("sdy", sdy), ("wqT", wqT), ("sw", sw), ("dx", dx),
+                    ("workspace", workspace)], stream)
     _record(stream, [dx] if allocated else [])
     _check(lib.fp8_block_gemm_dgrad(_ptr(dyq), _ptr(sdy), _ptr(wqT), _ptr(sw), _ptr(dx), M, N, K,
-                                    _stream(stream)),
+                                    *_workspace(workspace), _stream(stream)),
            "fp8_block_gemm_dgrad")
     return dx
 
 
-def fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=None, stream=None):
+def fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=None, stream=None, workspace=None):
     """dW[N, K] = dY^T X (bf16) from along-token codes: dY^T [N, M] / scales
     [M/128, N] and X^T [K, M] / scales [M/128, K]."""
     lib = load()
@@ -292,15 +324,16 @@ def fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=None, stream=None):
     _want(sxT, torch.float32, (M // 128, K), "sxT")
     allocated = dw is None
     dw = _out(dw, torch.bfloat16, (N, K), dyqT.device, "dw")
-    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw)], stream)
+    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw),
+                    ("workspace", workspace)], stream)
     _record(stream, [dw] if allocated else [])
     _check(lib.fp8_block_gemm_wgrad(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw), N, K, M,
-                                    _stream(stream)),
+                                    *_workspace(workspace), _stream(stream)),
            "fp8_block_gemm_wgrad")
     return dw
 
 
-def fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, stream=None):
+def fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, stream=None, workspace=None):
     """dW[N, K] += dY^T X in FP32, in place, from the same along-token codes
     as fp8_block_gemm_wgrad; dw is a float32 [N, K] tensor (the main
     gradient).  Returns dw."""
@@ -312,9 +345,10 @@ def fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, stream=None):
     _want(xqT, torch.uint8, (K, M), "xqT")
     _want(sxT, torch.float32, (M // 128, K), "sxT")
     _want(dw, torch.float32, (N, K), "dw")
-    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw)], stream)
+    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw),
+                    ("workspace", workspace)], stream)
     _check(lib.fp8_block_gemm_wgrad_accum_f32(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw),
-                                              N, K, M, _stream(stream)),
+                                              N, K, M, *_workspace(workspace), _stream(stream)),
            "fp8_block_gemm_wgrad_accum_f32")
     return dw
 
@@ -383,3 +417,20 @@ def fp8_selftest_silu_bf16(stream=None):
     _check(load().fp8_selftest_silu_bf16(_ptr(out), _stream(stream)), "fp8_selftest_silu_bf16")
     torch.cuda.synchronize()
     return out.cpu().numpy().view("uint16")
+
+
+def fp8_selftest_gemm_schedule(M: int, N: int, K: int, pairs: int, split: bool):
+    """The GEMMs' work schedule as the library computes it (host code shared
+    with the kernel): a list of (pair, tile, kb0, kb1, add_first, add_end)."""
+    import numpy as np
+
+    cap = 1 << 16
+    rows = np.zeros((cap, 5), dtype=np.int32)
+    n = ctypes.c_int64(0)
+    _check(load().fp8_selftest_gemm_schedule(int(M), int(N), int(K), int(pairs), int(bool(split)),
+                                            ctypes.c_void_p(rows.ctypes.data), cap, ctypes.byref(n)),
+           "fp8_selftest_gemm_schedule")
+    out = []
+    for r in rows[: n.value]:
+        out.append((int(r[0]), int(r[1]), int(r[2]), int(r[3]), int(r[4]) >> 16, int(r[4]) & 0xFFFF))
+    return out

@@ -214,11 +214,31 @@ fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t*
     return last_launch_status("tile quantize launch");
 }
 
+// Workspace of the split schedule for `pairs` CTA pairs: FP32 partial sums
+// [pairs][2][EPI_WARPS][128][32], then one flag per pair, CTA and warp.
+constexpr size_t kPartialFloatsPerPair = size_t(2) * gemm::EPI_WARPS * 128 * 32;
+inline size_t gemm_workspace_bytes(int pairs) {
+    const size_t partial = size_t(pairs) * kPartialFloatsPerPair * sizeof(float);
+    const size_t flags = size_t(pairs) * 2 * gemm::EPI_WARPS * sizeof(int);
+    return (partial + flags + 255) / 256 * 256;
+}
+
+// Whole tiles round-robin for all waves but the last two when the last wave
+// would leave more than 5% of the pairs idle; those tiles are then cut into
+// ranges of slabs of equal length, one per pair.
+inline int dp_tiles_for(int64_t tiles, int pairs) {
+    const int64_t waves = (tiles + pairs - 1) / pairs;
+    if (tiles >= waves * pairs * 95 / 100) return static_cast<int>(tiles);
+    const int64_t full = tiles / pairs;
+    return static_cast<int>(full >= 1 ? (full - 1) * pairs : 0);
+}
+
 // Shared launcher of the GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
 // codes, both K-major; scales described by `p`; out: [M_out, N_out] BF16, or
 // FP32 added to in place (OUT == kOutAccF32).
 template <int SCALE, int OUT>
-fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Params p, cudaStream_t stream) {
+fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Params p, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
     int dev = 0, sms = 0;
     fp8_status st = current_device(&dev);
     if (st != FP8_OK) return st;
@@ -259,7 +279,19 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Para
     p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     p.stall_tx = take_stall(1);
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-    const int grid = 2 * static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    p.dp_tiles = static_cast<int>(tiles);
+    p.ws_partial = nullptr;
+    p.ws_flags = nullptr;
+    if (workspace && workspace_bytes >= gemm_workspace_bytes(max_pairs) && p.K / gemm::BK > 1)
+        p.dp_tiles = dp_tiles_for(tiles, max_pairs);
+    int grid_pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    if (p.dp_tiles < tiles) {
+        grid_pairs = max_pairs;
+        p.ws_partial = static_cast<float*>(workspace);
+        p.ws_flags = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
+                                            size_t(max_pairs) * kPartialFloatsPerPair * sizeof(float));
+    }
+    const int grid = 2 * grid_pairs;
     const cudaError_t e = launch_pdl(gemm::gemm_kernel<SCALE, OUT>, dim3(grid), dim3(gemm::THREADS),
                                      gemm::SMEM_BYTES, stream, ma, mb, mc, p);
     if (e != cudaSuccess) return cuda_fail("gemm launch", e);
@@ -366,11 +398,12 @@ fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k,
 
 fp8_status fp8_block_gemm_fprop(const uint8_t* xq, const float* sx, const uint8_t* wq,
                                 const float* sw, void* y_bf16, int64_t M, int64_t N, int64_t K,
-                                void* stream) {
+                                void* workspace, size_t workspace_bytes, void* stream) {
     if (!dims_ok_gemm(M, N, K, false) || K > FP8_MAX_CONTRACTION_FPROP) return FP8_ERR_SHAPE;
     if (M == 0) return FP8_OK;
     if (!xq || !sx || !wq || !sw || !y_bf16) return FP8_ERR_NULL;
-    if (!aligned16(xq) || !aligned16(sx) || !aligned16(wq) || !aligned16(sw) || !aligned16(y_bf16))
+    if (!aligned16(xq) || !aligned16(sx) || !aligned16(wq) || !aligned16(sw) || !aligned16(y_bf16) ||
+        !aligned16(workspace))
         return FP8_ERR_ALIGN;
     gemm::Params p{};
     p.sa = sx;
@@ -381,16 +414,18 @@ fp8_status fp8_block_gemm_fprop(const uint8_t* xq, const float* sx, const uint8_
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
-    return launch_gemm<gemm::kScaleRowBlock, gemm::kOutBf16>(xq, wq, y_bf16, p, static_cast<cudaStream_t>(stream));
+    return launch_gemm<gemm::kScaleRowBlock, gemm::kOutBf16>(xq, wq, y_bf16, p, workspace, workspace_bytes,
+                                                             static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_dgrad(const uint8_t* dyq, const float* sdy, const uint8_t* wqT,
                                 const float* sw, void* dx_bf16, int64_t M, int64_t N, int64_t K,
-                                void* stream) {
+                                void* workspace, size_t workspace_bytes, void* stream) {
     if (!dims_ok_gemm(M, K, N, false) || N > FP8_MAX_CONTRACTION_FPROP) return FP8_ERR_SHAPE;
     if (M == 0) return FP8_OK;
     if (!dyq || !sdy || !wqT || !sw || !dx_bf16) return FP8_ERR_NULL;
-    if (!aligned16(dyq) || !aligned16(sdy) || !aligned16(wqT) || !aligned16(sw) || !aligned16(dx_bf16))
+    if (!aligned16(dyq) || !aligned16(sdy) || !aligned16(wqT) || !aligned16(sw) || !aligned16(dx_bf16) ||
+        !aligned16(workspace))
         return FP8_ERR_ALIGN;
     gemm::Params p{};
     p.sa = sdy;
@@ -401,29 +436,55 @@ fp8_status fp8_block_gemm_dgrad(const uint8_t* dyq, const float* sdy, const uint
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(K);
     p.K = static_cast<int>(N);
-    return launch_gemm<gemm::kScaleRowBlock, gemm::kOutBf16>(dyq, wqT, dx_bf16, p, static_cast<cudaStream_t>(stream));
+    return launch_gemm<gemm::kScaleRowBlock, gemm::kOutBf16>(dyq, wqT, dx_bf16, p, workspace, workspace_bytes,
+                                                             static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_wgrad(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
                                 const float* sxT, void* dw_bf16, int64_t N, int64_t K, int64_t M,
-                                void* stream) {
+                                void* workspace, size_t workspace_bytes, void* stream) {
     if (!dims_ok_gemm(N, K, M, true)) return FP8_ERR_SHAPE;
     if (!dyqT || !sdyT || !xqT || !sxT || !dw_bf16) return FP8_ERR_NULL;
-    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_bf16))
+    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_bf16) ||
+        !aligned16(workspace))
         return FP8_ERR_ALIGN;
     return launch_gemm<gemm::kScaleOuter, gemm::kOutBf16>(dyqT, xqT, dw_bf16, wgrad_params(sdyT, sxT, N, K, M),
-                                                          static_cast<cudaStream_t>(stream));
+                                                          workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
                                           const float* sxT, float* dw_f32, int64_t N, int64_t K, int64_t M,
-                                          void* stream) {
+                                          void* workspace, size_t workspace_bytes, void* stream) {
     if (!dims_ok_gemm(N, K, M, true)) return FP8_ERR_SHAPE;
     if (!dyqT || !sdyT || !xqT || !sxT || !dw_f32) return FP8_ERR_NULL;
-    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_f32))
+    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_f32) ||
+        !aligned16(workspace))
         return FP8_ERR_ALIGN;
     return launch_gemm<gemm::kScaleOuter, gemm::kOutAccF32>(dyqT, xqT, dw_f32, wgrad_params(sdyT, sxT, N, K, M),
+                                                            workspace, workspace_bytes,
                                                             static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_gemm_workspace_bytes(size_t* bytes) {
+    if (!bytes) return FP8_ERR_NULL;
+    int dev = 0;
+    fp8_status st = current_device(&dev);
+    if (st != FP8_OK) return st;
+    int pairs = 0;
+    // Resident CTA pairs of the GEMM kernels (all variants share one shape).
+    cudaLaunchConfig_t cfg = {};
+    int sms = 0;
+    if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
+    cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<gemm::kScaleRowBlock, gemm::kOutBf16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
+    cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+    cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
+    e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<gemm::kScaleRowBlock, gemm::kOutBf16>, &cfg);
+    if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
+    *bytes = gemm_workspace_bytes(pairs);
+    return FP8_OK;
 }
 
 fp8_status fp8_get_error(void) {
@@ -487,6 +548,49 @@ fp8_status fp8_selftest_silu_bf16(uint16_t* out, void* stream) {
     if (!aligned16(out)) return FP8_ERR_ALIGN;
     silu_selftest_kernel<<<256, 256, 0, static_cast<cudaStream_t>(stream)>>>(out);
     return last_launch_status("silu self-test launch");
+}
+
+fp8_status fp8_selftest_gemm_schedule(int64_t M, int64_t N, int64_t K, int pairs, int split, int32_t* segs,
+                                      int64_t max_segs, int64_t* nsegs) {
+    if (!segs || !nsegs) return FP8_ERR_NULL;
+    if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 128 || pairs <= 0 || max_segs < 0 ||
+        M > kMaxDim || N > kMaxDim || K > kMaxDim)
+        return FP8_ERR_SHAPE;
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.tiles_m = static_cast<int>((M + 2 * gemm::BM - 1) / (2 * gemm::BM));
+    p.tiles_n = static_cast<int>((N + gemm::BN - 1) / gemm::BN);
+    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    p.dp_tiles = (split && p.K / gemm::BK > 1) ? dp_tiles_for(tiles, pairs) : static_cast<int>(tiles);
+    const int npairs = p.dp_tiles < tiles ? pairs : static_cast<int>(tiles < pairs ? tiles : pairs);
+    int64_t n = 0;
+    for (int q = 0; q < npairs; ++q) {
+        gemm::Schedule sch(p, q, npairs);
+        gemm::Seg sg;
+        while (sch.next(sg)) {
+            if (n >= max_segs) return FP8_ERR_SHAPE;
+            int32_t* row = segs + 5 * n;
+            row[0] = q;
+            row[1] = sg.tile;
+            row[2] = sg.kb0;
+            row[3] = sg.kb1;
+            // the pairs whose partial sums a finalizing segment adds: the
+            // first and one past the last (equal when none)
+            int32_t first = 0, last = 0;
+            if (sg.kb0 == 0 && sg.kb1 < sch.num_kb) {
+                const int64_t tile_end = static_cast<int64_t>(sg.tile + 1) * sch.num_kb - sch.sk_base;
+                first = q + 1;
+                last = q + 1;
+                for (int r = q + 1; r < npairs && sch.range_begin(r) < tile_end; ++r) last = r + 1;
+            }
+            row[4] = (first << 16) | last;
+            ++n;
+        }
+    }
+    *nsegs = n;
+    return FP8_OK;
 }
 
 fp8_status fp8_selftest_stall_next(int which) {

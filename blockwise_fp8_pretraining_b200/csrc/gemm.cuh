@@ -132,7 +132,70 @@ struct Params {
     uint64_t wait_ns;
     uint32_t stall_tx;      // test only: extra bytes the first stage's barrier expects (0 normally)
     float* out_f32;         // main-gradient mode: the FP32 array [M, N] added to
+    // Split schedule (see Schedule): tiles [0, dp_tiles) whole, the rest as
+    // contiguous ranges of (tile, slab) units, partial sums through
+    // ws_partial [pairs][2][EPI_WARPS][128][32] f32 and ws_flags
+    // [pairs][2][EPI_WARPS] (zero between calls).  dp_tiles == total tiles
+    // means no split (the workspace is then unused and may be null).
+    int dp_tiles;
+    float* ws_partial;
+    int* ws_flags;
 };
+
+// The work of one CTA pair: first its share of whole tiles (tile = pair,
+// pair + npairs, ... below dp_tiles), then one contiguous range of units
+// (unit = tile * num_kb + slab) over the remaining tiles, cut evenly across
+// the pairs so that the last wave has no idle pairs.  A range cuts tiles into
+// segments of slabs: a segment that starts inside a tile leaves its FP32
+// partial sums to the pair whose segment holds the tile's first slab, which
+// adds them before the epilogue.  Every partial segment is the first segment
+// of its pair's range, so a pair never waits for a partial before it has
+// written its own, and no wait can be circular.
+struct Seg {
+    int tile, kb0, kb1;
+};
+
+struct Schedule {
+    int num_kb, dp_tiles, npairs, next_dp;
+    int64_t u, u_end, sk_base, sk_units;
+    __host__ __device__ __forceinline__ Schedule(const Params& p, int pair, int npairs_)
+        : num_kb(p.K / BK), dp_tiles(p.dp_tiles), npairs(npairs_), next_dp(pair) {
+        const int total = p.tiles_m * p.tiles_n;
+        sk_base = static_cast<int64_t>(dp_tiles) * num_kb;
+        sk_units = static_cast<int64_t>(total - dp_tiles) * num_kb;
+        u = sk_base + range_begin(pair);
+        u_end = sk_base + range_begin(pair + 1);
+    }
+    // First unit (relative to sk_base) of pair q's range.
+    __host__ __device__ __forceinline__ int64_t range_begin(int q) const { return sk_units * q / npairs; }
+    __host__ __device__ __forceinline__ bool next(Seg& sg) {
+        if (next_dp < dp_tiles) {
+            sg.tile = next_dp;
+            sg.kb0 = 0;
+            sg.kb1 = num_kb;
+            next_dp += npairs;
+            return true;
+        }
+        if (u >= u_end) return false;
+        sg.tile = static_cast<int>(u / num_kb);
+        sg.kb0 = static_cast<int>(u - static_cast<int64_t>(sg.tile) * num_kb);
+        const int64_t left = u_end - u;
+        const int64_t end = sg.kb0 + left;
+        sg.kb1 = static_cast<int>(end < num_kb ? end : num_kb);
+        u += sg.kb1 - sg.kb0;
+        return true;
+    }
+};
+
+// Release / acquire flag accesses for the partial-sum hand-over between pairs.
+__device__ __forceinline__ void st_release_gpu(int* addr, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    return v;
+}
 
 struct Bars {
     uint32_t full, empty, tfull, tempty, sfull, sempty, drain;
@@ -160,8 +223,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t rank = cluster_ctarank();            // 0 = leader of the pair
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
-    const int num_kb = p.K / BK;
-    const int total_tiles = p.tiles_m * p.tiles_n;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
 
     Bars bars;
@@ -214,10 +275,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const uint32_t full_leader = map_to_cta(bars.full, 0);
             int it = 0;    // slabs whose operand tiles were requested
             bool ok = true;
-            for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-                const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
-                const int n0 = (tile % p.tiles_n) * BN;
-                for (int kb = 0; kb < num_kb; ++kb) {
+            Schedule sch(p, pair, npairs);
+            Seg sg;
+            while (ok && sch.next(sg)) {
+                const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
+                const int n0 = (sg.tile % p.tiles_n) * BN;
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     const int s = it % STAGES;
                     if (!mbar_wait(bars.empty_(s), ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout,
                                    kProducerSleepNs)) {
@@ -249,14 +312,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // bulk copy) and store them into the slot before lane 0 arrives.
         int ic = 0;    // scale chunks requested
         bool ok = true;
-        for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-            const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
-            const int n0 = (tile % p.tiles_n) * BN;
+        Schedule sch(p, pair, npairs);
+        Seg sg;
+        while (ok && sch.next(sg)) {
+            const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
+            const int n0 = (sg.tile % p.tiles_n) * BN;
             const uint32_t sa_bytes = (m_own < p.M) ? BM * 4u : 0u;
             const uint32_t sb_bytes =
                 (SCALE == kScaleOuter) ? static_cast<uint32_t>(min(BN, p.N - n0)) * 4u : 0u;
-            for (int kb0 = 0; kb0 < num_kb; kb0 += SCHUNK) {
-                const int nslab = min(SCHUNK, num_kb - kb0);
+            for (int kb0 = sg.kb0; kb0 < sg.kb1; kb0 += SCHUNK) {
+                const int nslab = min(SCHUNK, sg.kb1 - kb0);
                 const int sl = ic % SSLOTS;
                 const bool got = mbar_wait(bars.sempty_(sl), ((ic / SSLOTS) & 1) ^ 1, abort_flag, p.wait_ns,
                                            kErrTimeout, kScaleSleepNs);
@@ -302,8 +367,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int sel = (warp == 1) ? 0 : 1;
             int it = 0;
             bool ok = true;
-            for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            Schedule sch(p, pair, npairs);
+            Seg sg;
+            while (ok && sch.next(sg)) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                     if ((it & 1) != sel) continue;
                     const int buf = it & 1;
                     if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout,
@@ -351,16 +418,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         int it = 0;
         int ic = 0;        // scale chunks consumed
         bool ok = true;
-        for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-            const int m_own = (tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
-            const int n0 = (tile % p.tiles_n) * BN;
+        Schedule sch(p, pair, npairs);
+        Seg sg;
+        while (ok && sch.next(sg)) {
+            const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
+            const int n0 = (sg.tile % p.tiles_n) * BN;
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                 const int buf = it & 1;
                 const int sl = ic % SSLOTS;
-                const int j_in_chunk = kb % SCHUNK;
+                const int j_in_chunk = (kb - sg.kb0) % SCHUNK;
                 bool got = true;
                 if (j_in_chunk == 0)
                     got = mbar_wait(bars.sfull_(sl), (ic / SSLOTS) & 1, abort_flag, p.wait_ns, kErrTimeout);
@@ -428,7 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
                 promote(ra, 64);
                 promote(rb, 96);
-                if (j_in_chunk == SCHUNK - 1 || kb == num_kb - 1) {
+                if (j_in_chunk == SCHUNK - 1 || kb == sg.kb1 - 1) {
                     // last slab of this scale chunk: the slot may be refilled
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bars.sempty_(sl));
@@ -436,6 +505,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
             if (!ok) break;
+
+            if (sg.kb0 > 0) {
+                // A later part of a split tile: leave the partial sums to the
+                // pair that holds the tile's first slab.  Lane-fastest layout,
+                // so each store of the warp covers 128 contiguous bytes.
+                float* dst = p.ws_partial + ((static_cast<int64_t>(pair) * 2 + rank) * EPI_WARPS + ew) * (128 * 32);
+#pragma unroll
+                for (int j = 0; j < 128; ++j) __stcg(dst + j * 32 + lane, acc[j]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(p.ws_flags + (pair * 2 + rank) * EPI_WARPS + ew, 1);
+                continue;
+            }
+            if (sg.kb1 < sch.num_kb) {
+                // The first part of a split tile: add the partial sums of the
+                // pairs holding the rest, in pair order, then the epilogue.
+                // (A pair with an empty range holds nothing.)
+                const int64_t tile_end = static_cast<int64_t>(sg.tile + 1) * sch.num_kb - sch.sk_base;
+                for (int q = pair + 1; q < npairs && sch.range_begin(q) < tile_end; ++q) {
+                    if (sch.range_begin(q) == sch.range_begin(q + 1)) continue;
+                    const int* flag = p.ws_flags + (q * 2 + rank) * EPI_WARPS + ew;
+                    const uint64_t t0 = globaltimer_ns();
+                    bool got = true;
+                    while (ld_acquire_gpu(flag) == 0) {
+                        if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
+                            if (!*abort_flag) {
+                                record_error(kErrTimeout);
+                                *abort_flag = 1;
+                            }
+                            got = false;
+                            break;
+                        }
+                    }
+                    if (!__all_sync(0xffffffffu, got)) {
+                        ok = false;
+                        break;
+                    }
+                    const float* src = p.ws_partial + ((static_cast<int64_t>(q) * 2 + rank) * EPI_WARPS + ew) * (128 * 32);
+#pragma unroll
+                    for (int j = 0; j < 128; ++j) acc[j] += __ldcg(src + j * 32 + lane);
+                    __syncwarp();
+                    if (lane == 0) *const_cast<volatile int*>(flag) = 0;     // zero again for the next call
+                }
+                if (!ok) break;
+            }
 
             // BF16 round-to-nearest-even into this warp's staging buffer (two
             // 32 x 64 boxes, 128-byte rows, 16-byte chunk j of row r at

@@ -58,6 +58,7 @@
 #ifndef FP8BLK_H
 #define FP8BLK_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -85,6 +86,27 @@ enum {
 /* Largest contraction length (K of fprop, N of dgrad) the fprop/dgrad GEMMs
  * accept: 256 slabs of 128. */
 #define FP8_MAX_CONTRACTION_FPROP 32768
+
+/*
+ * GEMM workspace.  Every GEMM entry point takes an optional device
+ * workspace (workspace, workspace_bytes; NULL and 0 to go without).  With
+ * one of at least fp8_gemm_workspace_bytes() bytes, a GEMM whose last wave
+ * of 256x256 output tiles would leave more than 5% of the GPU's CTA pairs
+ * idle cuts the tiles of its last two waves into equal ranges of 128-wide
+ * contraction slabs, one range per pair; the pair holding a tile's first
+ * slab adds the FP32 partial sums the other pairs leave in the workspace
+ * (in a fixed order, so results are reproducible run to run) before its
+ * epilogue.  Without a workspace every tile is computed whole by one pair.
+ * Either way every output element satisfies the same error bound.
+ *
+ * The workspace is owned by the caller, 16-byte aligned, and must hold
+ * zeros before its first use (cudaMemset); every call that completes leaves
+ * it zeroed again.  After a call that reported FP8_ERR_TIMEOUT it must be
+ * zeroed before reuse.  Two launches that may run at the same time (on
+ * different streams) need different workspaces.  The size depends on the
+ * device (about 19 MB on a 148-SM B200).
+ */
+fp8_status fp8_gemm_workspace_bytes(size_t *bytes);
 
 /*
  * Activation quantizer, 1x128 groups (row-wise) and/or 128x1 groups along
@@ -160,10 +182,12 @@ fp8_status fp8_quantize_weight_128x128(const void *w_bf16, int64_t n, int64_t k,
  *   M >= 0, a multiple of 128; N > 0 and K > 0, multiples of 128;
  *   K <= FP8_MAX_CONTRACTION_FPROP.  M == 0 is a no-op (pointers may then
  *   be NULL).
+ *   workspace, workspace_bytes: see "GEMM workspace" above.
  */
 fp8_status fp8_block_gemm_fprop(const uint8_t *xq, const float *sx, const uint8_t *wq,
                                 const float *sw, void *y_bf16, int64_t M, int64_t N,
-                                int64_t K, void *stream);
+                                int64_t K, void *workspace, size_t workspace_bytes,
+                                void *stream);
 
 /*
  * dgrad: dX[m, k] = sum_n dY[m, n] W[n, k]   (dX = dY W), BF16 out.
@@ -182,10 +206,12 @@ fp8_status fp8_block_gemm_fprop(const uint8_t *xq, const float *sx, const uint8_
  *   M >= 0, a multiple of 128; N > 0 and K > 0, multiples of 128;
  *   N <= FP8_MAX_CONTRACTION_FPROP.  M == 0 is a no-op (pointers may then
  *   be NULL).
+ *   workspace, workspace_bytes: see "GEMM workspace" above.
  */
 fp8_status fp8_block_gemm_dgrad(const uint8_t *dyq, const float *sdy, const uint8_t *wqT,
                                 const float *sw, void *dx_bf16, int64_t M, int64_t N,
-                                int64_t K, void *stream);
+                                int64_t K, void *workspace, size_t workspace_bytes,
+                                void *stream);
 
 /*
  * wgrad: dW[n, k] = sum_m dY[m, n] X[m, k]   (dW = dY^T X), contracting over
@@ -199,10 +225,12 @@ fp8_status fp8_block_gemm_dgrad(const uint8_t *dyq, const float *sdy, const uint
  *   xqT  [K, M] u8, sxT  [M/128, K] f32 - column-wise (along-token) X
  *   dw_bf16 [N, K]
  *   M > 0, N > 0, K > 0, all multiples of 128.
+ *   workspace, workspace_bytes: see "GEMM workspace" above.
  */
 fp8_status fp8_block_gemm_wgrad(const uint8_t *dyqT, const float *sdyT, const uint8_t *xqT,
                                 const float *sxT, void *dw_bf16, int64_t N, int64_t K,
-                                int64_t M, void *stream);
+                                int64_t M, void *workspace, size_t workspace_bytes,
+                                void *stream);
 
 /*
  * wgrad accumulated into an FP32 main gradient: dW_f32[n, k] += sum_m
@@ -215,13 +243,16 @@ fp8_status fp8_block_gemm_wgrad(const uint8_t *dyqT, const float *sdyT, const ui
  * of one optimizer step follows from the setting table (global batch 1536,
  * micro-batch 2).
  *
- *   dyqT, sdyT, xqT, sxT, N, K, M - as fp8_block_gemm_wgrad
+ *   dyqT, sdyT, xqT, sxT, N, K, M, workspace, workspace_bytes - as
+ *          fp8_block_gemm_wgrad
  *   dw_f32 [N, K] f32, read and written (16-byte aligned); must not overlap
  *          the inputs.  Calls on the same dw_f32 must be ordered (one stream).
+ *          A sum below float32's normal range may be flushed to zero.
  */
 fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t *dyqT, const float *sdyT,
                                           const uint8_t *xqT, const float *sxT,
                                           float *dw_f32, int64_t N, int64_t K, int64_t M,
+                                          void *workspace, size_t workspace_bytes,
                                           void *stream);
 
 /* Sticky per-device error word: FP8_OK, or the first FP8_ERR_TIMEOUT a
@@ -273,6 +304,18 @@ fp8_status fp8_selftest_wait_timeout(void *stream);
  * checking it exhaustively).  out: 65536 device uint16, 16-byte aligned.
  * Non-finite g are outside the definition. */
 fp8_status fp8_selftest_silu_bf16(uint16_t *out, void *stream);
+
+/* The GEMMs' work schedule, computed on the host by the same code the
+ * kernel runs, for checking without a GPU: for an output of M x N over a
+ * contraction of K, with `pairs` CTA pairs and split != 0 meaning "with a
+ * workspace", writes one row of 5 int32 per segment of work, pair by pair
+ * in execution order: pair, tile, first slab, one past the last slab, and
+ * (first << 16 | end) of the range of pairs whose partial sums the segment
+ * adds before its epilogue (first == end when none).  max_segs rows fit in
+ * segs; *nsegs receives the count.  FP8_ERR_SHAPE for bad sizes or too many
+ * segments. */
+fp8_status fp8_selftest_gemm_schedule(int64_t M, int64_t N, int64_t K, int pairs, int split,
+                                      int32_t *segs, int64_t max_segs, int64_t *nsegs);
 
 /* Arms the next launch of a kernel family so that the first operand
  * barrier of every CTA (pair) expects 16 bytes more than its copies bring:

@@ -34,6 +34,18 @@ def dev():
     return torch.device("cuda", torch.cuda.current_device())
 
 
+_WORKSPACES = {}
+
+
+def workspace():
+    """The tests' GEMM workspace on the current device (zeroed once; every
+    completed GEMM leaves it zeroed).  The tests launch one GEMM at a time."""
+    d = torch.cuda.current_device()
+    if d not in _WORKSPACES:
+        _WORKSPACES[d] = fp8.fp8_gemm_workspace()
+    return _WORKSPACES[d]
+
+
 def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
@@ -122,13 +134,13 @@ def pick_rows(total: int, count: int, seed: int) -> np.ndarray:
     return rows
 
 
-def check_fprop(x: torch.Tensor, w: torch.Tensor, rows=None, what="fprop", output_rounding=False):
+def check_fprop(x: torch.Tensor, w: torch.Tensor, rows=None, what="fprop", output_rounding=False, ws=None):
     """GPU: quantize + fprop through the C ABI; oracle: quantize + fprop on
     the selected rows (all when rows is None).  Returns the GPU output."""
     d = dev()
     xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x.to(d), fp8.ROWWISE)
     wq, sw, _ = fp8.fp8_quantize_weight_128x128(w.to(d), transposed=False)
-    y = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+    y = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, workspace=ws)
     torch.cuda.synchronize()
     xq_o, sx_o = oracle.quantize_act_rowwise(syn.bf16_bits(x))
     wq_o, sw_o = oracle.quantize_weight(syn.bf16_bits(w))
@@ -138,11 +150,11 @@ def check_fprop(x: torch.Tensor, w: torch.Tensor, rows=None, what="fprop", outpu
     return y
 
 
-def check_dgrad(dy: torch.Tensor, w: torch.Tensor, rows=None, what="dgrad", output_rounding=False):
+def check_dgrad(dy: torch.Tensor, w: torch.Tensor, rows=None, what="dgrad", output_rounding=False, ws=None):
     d = dev()
     dyq, sdy, _, _ = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.ROWWISE)
     _, sw, wqT = fp8.fp8_quantize_weight_128x128(w.to(d))
-    dx = fp8.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw)
+    dx = fp8.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, workspace=ws)
     torch.cuda.synchronize()
     dyq_o, sdy_o = oracle.quantize_act_rowwise(syn.bf16_bits(dy))
     wq_o, sw_o = oracle.quantize_weight(syn.bf16_bits(w))
@@ -152,11 +164,11 @@ def check_dgrad(dy: torch.Tensor, w: torch.Tensor, rows=None, what="dgrad", outp
     return dx
 
 
-def check_wgrad(dy: torch.Tensor, x: torch.Tensor, rows=None, what="wgrad", output_rounding=False):
+def check_wgrad(dy: torch.Tensor, x: torch.Tensor, rows=None, what="wgrad", output_rounding=False, ws=None):
     d = dev()
     _, _, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.COLWISE)
     _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
-    dw = fp8.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT)
+    dw = fp8.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, workspace=ws)
     torch.cuda.synchronize()
     dyqT_o, sdyT_o = oracle.quantize_act_colwise(syn.bf16_bits(dy))
     xqT_o, sxT_o = oracle.quantize_act_colwise(syn.bf16_bits(x))

@@ -82,29 +82,37 @@ def test_quantize_weight_rejections(lib):
 def test_fprop_dgrad_rejections(lib, name):
     g = getattr(lib, name)
     a = [P(A16)] * 5
-    assert g(*a, 100, 256, 256, S) == SHAPE          # M not a multiple of 128
-    assert g(*a, 128, 0, 256, S) == SHAPE
-    assert g(*a, 128, 256, 0, S) == SHAPE
-    assert g(*a, 128, 200, 256, S) == SHAPE
+    W = (None, 0)                                    # no workspace
+    assert g(*a, 100, 256, 256, *W, S) == SHAPE      # M not a multiple of 128
+    assert g(*a, 128, 0, 256, *W, S) == SHAPE
+    assert g(*a, 128, 256, 0, *W, S) == SHAPE
+    assert g(*a, 128, 200, 256, *W, S) == SHAPE
     big = fp8.MAX_CONTRACTION_FPROP + 128
     if name == "fp8_block_gemm_fprop":
-        assert g(*a, 128, 256, big, S) == SHAPE
+        assert g(*a, 128, 256, big, *W, S) == SHAPE
     else:
-        assert g(*a, 128, big, 256, S) == SHAPE
-    assert g(None, *a[1:], 128, 256, 256, S) == NULL
-    assert g(*a[:4], None, 128, 256, 256, S) == NULL
-    assert g(*a[:2], P(MIS), *a[3:], 128, 256, 256, S) == ALIGN
-    assert g(*a, 0, 256, 256, S) == OK               # M == 0: nothing to do
+        assert g(*a, 128, big, 256, *W, S) == SHAPE
+    assert g(None, *a[1:], 128, 256, 256, *W, S) == NULL
+    assert g(*a[:4], None, 128, 256, 256, *W, S) == NULL
+    assert g(*a[:2], P(MIS), *a[3:], 128, 256, 256, *W, S) == ALIGN
+    assert g(*a, 128, 256, 256, P(MIS), 1 << 30, S) == ALIGN     # misaligned workspace
+    assert g(*a, 0, 256, 256, *W, S) == OK           # M == 0: nothing to do
 
 
 def test_wgrad_rejections(lib):
     g = lib.fp8_block_gemm_wgrad
     a = [P(A16)] * 5
-    assert g(*a, 256, 256, 0, S) == SHAPE            # no tokens
-    assert g(*a, 256, 256, 100, S) == SHAPE
-    assert g(*a, 200, 256, 256, S) == SHAPE
-    assert g(*a[:3], None, a[4], 256, 256, 256, S) == NULL
-    assert g(*a[:4], P(MIS), 256, 256, 256, S) == ALIGN
+    W = (None, 0)
+    assert g(*a, 256, 256, 0, *W, S) == SHAPE        # no tokens
+    assert g(*a, 256, 256, 100, *W, S) == SHAPE
+    assert g(*a, 200, 256, 256, *W, S) == SHAPE
+    assert g(*a[:3], None, a[4], 256, 256, 256, *W, S) == NULL
+    assert g(*a[:4], P(MIS), 256, 256, 256, *W, S) == ALIGN
+    assert g(*a, 256, 256, 256, P(MIS), 1 << 30, S) == ALIGN
+
+
+def test_workspace_size_query_rejects_null(lib):
+    assert lib.fp8_gemm_workspace_bytes(None) == NULL
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
@@ -130,10 +138,11 @@ int main(void) {
     EXPECT(fp8_quantize_act_1x128(a16, 100, 256, FP8_COLWISE, NULL, NULL, u, f, NULL), FP8_ERR_SHAPE);
     EXPECT(fp8_quantize_act_1x128(NULL, 0, 256, FP8_BOTH, NULL, NULL, NULL, NULL, NULL), FP8_OK);
     EXPECT(fp8_quantize_weight_128x128(a16, 128, 200, u, f, NULL, NULL), FP8_ERR_SHAPE);
-    EXPECT(fp8_block_gemm_fprop(u, f, u, f, a16, 128, 128, FP8_MAX_CONTRACTION_FPROP + 128, NULL),
-           FP8_ERR_SHAPE);
-    EXPECT(fp8_block_gemm_dgrad(u, f, NULL, f, a16, 128, 128, 128, NULL), FP8_ERR_NULL);
-    EXPECT(fp8_block_gemm_wgrad(u, f, u, f, a16, 128, 128, 0, NULL), FP8_ERR_SHAPE);
+    EXPECT(fp8_block_gemm_fprop(u, f, u, f, a16, 128, 128, FP8_MAX_CONTRACTION_FPROP + 128, NULL, 0,
+                                NULL), FP8_ERR_SHAPE);
+    EXPECT(fp8_block_gemm_dgrad(u, f, NULL, f, a16, 128, 128, 128, NULL, 0, NULL), FP8_ERR_NULL);
+    EXPECT(fp8_block_gemm_wgrad(u, f, u, f, a16, 128, 128, 0, NULL, 0, NULL), FP8_ERR_SHAPE);
+    EXPECT(fp8_gemm_workspace_bytes(NULL), FP8_ERR_NULL);
     EXPECT(fp8_set_wait_timeout_ns(0), FP8_OK);
     if (strcmp(fp8_status_string(FP8_ERR_ALIGN), "pointer not 16-byte aligned") != 0) return 1;
     if (fp8_last_cuda_error()[0] != '\0') return 1;
@@ -169,10 +178,13 @@ def test_stall_switch_rejects_unknown_kernel_families(lib):
 
 def test_wgrad_accum_rejections(lib):
     g = lib.fp8_block_gemm_wgrad_accum_f32
-    assert g(P(A16), P(A16), P(A16), P(A16), P(A16), 128, 128, 0, S) == SHAPE      # no tokens
-    assert g(P(A16), P(A16), P(A16), P(A16), P(A16), 128, 100, 128, S) == SHAPE
-    assert g(P(A16), P(A16), P(A16), P(A16), None, 128, 128, 128, S) == NULL
-    assert g(P(A16), P(A16), P(A16), P(A16), P(MIS), 128, 128, 128, S) == ALIGN
+    a4 = [P(A16)] * 4
+    W = (None, 0)
+    assert g(*a4, P(A16), 128, 128, 0, *W, S) == SHAPE      # no tokens
+    assert g(*a4, P(A16), 128, 100, 128, *W, S) == SHAPE
+    assert g(*a4, None, 128, 128, 128, *W, S) == NULL
+    assert g(*a4, P(MIS), 128, 128, 128, *W, S) == ALIGN
+    assert g(*a4, P(A16), 128, 128, 128, P(MIS), 1 << 30, S) == ALIGN
 
 
 def test_swiglu_quantize_rejections(lib):

@@ -109,7 +109,7 @@ def test_fprop_marshalling(rec):
     y = _abi.fp8_block_gemm_fprop(xq, sx, wq, sw)
     name, a = _args(rec)
     assert name == "fp8_block_gemm_fprop"
-    assert a == [p(xq), p(sx), p(wq), p(sw), p(y), M, N, K, STREAM]
+    assert a == [p(xq), p(sx), p(wq), p(sw), p(y), M, N, K, 0, 0, STREAM]
     assert y.shape == (M, N) and y.dtype == torch.bfloat16
     with pytest.raises(ValueError):        # scales in the other layout
         _abi.fp8_block_gemm_fprop(xq, sx.T.contiguous(), wq, sw)
@@ -124,7 +124,7 @@ def test_dgrad_marshalling(rec):
     dx = _abi.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw)
     name, a = _args(rec)
     assert name == "fp8_block_gemm_dgrad"
-    assert a == [p(dyq), p(sdy), p(wqT), p(sw), p(dx), M, N, K, STREAM]
+    assert a == [p(dyq), p(sdy), p(wqT), p(sw), p(dx), M, N, K, 0, 0, STREAM]
     assert dx.shape == (M, K)
 
 
@@ -137,7 +137,7 @@ def test_wgrad_marshalling(rec):
     dw = _abi.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT)
     name, a = _args(rec)
     assert name == "fp8_block_gemm_wgrad"
-    assert a == [p(dyqT), p(sdyT), p(xqT), p(sxT), p(dw), N, K, M, STREAM]
+    assert a == [p(dyqT), p(sdyT), p(xqT), p(sxT), p(dw), N, K, M, 0, 0, STREAM]
     assert dw.shape == (N, K)
 
 
@@ -173,3 +173,24 @@ def test_tensors_on_another_device_are_rejected():
         _abi._check_devices([("a", on(1)), ("b", on(0))], current=1)
     with pytest.raises(ValueError, match="current CUDA device is cuda:0"):
         _abi._check_devices([("x", on(3))], current=0)
+
+
+def test_gemm_workspace_marshalling(rec, monkeypatch):
+    """An optional workspace tensor goes over as (pointer, bytes) right
+    before the stream; a non-contiguous one is refused."""
+    monkeypatch.setattr(torch.Tensor, "is_cuda", property(lambda self: True))
+    N, K, M = 256, 128, 256
+    dyqT = torch.zeros((N, M), dtype=torch.uint8)
+    sdyT = torch.zeros((M // 128, N))
+    xqT = torch.zeros((K, M), dtype=torch.uint8)
+    sxT = torch.zeros((M // 128, K))
+    dw = torch.zeros((N, K))
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    _abi.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, workspace=ws)
+    name, a = _args(rec)
+    assert name == "fp8_block_gemm_wgrad_accum_f32"
+    assert a == [p(dyqT), p(sdyT), p(xqT), p(sxT), p(dw), N, K, M, p(ws), 4096, STREAM]
+    assert "workspace" in rec.checked[-1]
+    with pytest.raises(ValueError):
+        _abi.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw,
+                                            workspace=torch.zeros((64, 64), dtype=torch.uint8)[:, ::2])

@@ -1,5 +1,6 @@
 """GPU parity at the Qwen3-1.7B layer shapes (8192 tokens per micro-batch),
-launched exactly as the benchmark launches them.  Quantization is compared
+launched exactly as the benchmark launches them (GEMMs with a workspace, so
+that shapes with a partly idle last wave run the split schedule).  Quantization is compared
 bit for bit in full everywhere.  GEMM outputs of the attention-projection,
 SwiGLU-MLP and backward configurations are compared element by element in
 full; the 28-layer sweep compares a stratified seeded row sample per GEMM
@@ -16,6 +17,7 @@ Configurations:
                          wgrad (contraction over the 8192 tokens)
   28-layer sweep         every linear of every layer (seeds 0..27):
                          quantizers in full, GEMMs on the stratified rows
+                         (even layers with the split schedule, odd without)
   heavy tails            Student-t(3) with 0.1% of values x1e3, seeds 0..27,
                          quantizers in full
 """
@@ -29,8 +31,8 @@ import blockwise_fp8_pretraining_b200 as fp8
 import oracle
 from blockwise_fp8_pretraining_b200 import synthetic as syn
 
-from _parity import (assert_bits_equal, assert_within_bound, check_act, check_dgrad, check_fprop, check_wgrad,
-                     check_weight, dev, pick_rows)
+from _parity import (assert_bits_equal, assert_within_bound, check_act, check_dgrad, check_fprop,
+                     check_wgrad, check_weight, dev, pick_rows, workspace)
 
 pytestmark = pytest.mark.gpu
 
@@ -52,8 +54,8 @@ def test_attention_projections_fprop():
     check_act(c["x"], fp8.BOTH)
     check_weight(c["w_qkv"])
     check_weight(c["w_o"])
-    check_fprop(c["x"], c["w_qkv"], None, "qkv fprop")
-    check_fprop(c["x"], c["w_o"], None, "o_proj fprop")
+    check_fprop(c["x"], c["w_qkv"], None, "qkv fprop", ws=workspace())
+    check_fprop(c["x"], c["w_o"], None, "o_proj fprop", ws=workspace())
 
 
 def test_attention_projections_backward():
@@ -61,10 +63,10 @@ def test_attention_projections_backward():
     dy_qkv, dy_o = syn.output_grads([(syn.TOKENS, syn.QKV_OUT), (syn.TOKENS, syn.HIDDEN)], seed=1)
     check_act(dy_qkv, fp8.BOTH)
     check_act(dy_o, fp8.BOTH)
-    check_dgrad(dy_qkv, c["w_qkv"], None, "qkv dgrad")
-    check_dgrad(dy_o, c["w_o"], None, "o_proj dgrad")
-    check_wgrad(dy_qkv, c["x"], None, "qkv wgrad")
-    check_wgrad(dy_o, c["x"], None, "o_proj wgrad")
+    check_dgrad(dy_qkv, c["w_qkv"], None, "qkv dgrad", ws=workspace())
+    check_dgrad(dy_o, c["w_o"], None, "o_proj dgrad", ws=workspace())
+    check_wgrad(dy_qkv, c["x"], None, "qkv wgrad", ws=workspace())
+    check_wgrad(dy_o, c["x"], None, "o_proj wgrad", ws=workspace())
 
 
 @pytest.mark.slow
@@ -76,7 +78,7 @@ def test_swiglu_mlp_fprop():
     d = dev()
     xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x.to(d), fp8.ROWWISE)
     wq, sw, _ = fp8.fp8_quantize_weight_128x128(w_gu.to(d), transposed=False)
-    gu_gpu = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw)
+    gu_gpu = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, workspace=workspace())
     torch.cuda.synchronize()
     # the oracle's full gate_up output: every element compared, then H from it
     xq_o, sx_o = oracle.quantize_act_rowwise(syn.bf16_bits(x))
@@ -103,7 +105,7 @@ def test_swiglu_mlp_fprop():
     h = syn.swiglu_bf16(gu_b)
     del gu_b
     check_act(h, fp8.BOTH)
-    check_fprop(h, w_down, None, "down fprop")
+    check_fprop(h, w_down, None, "down fprop", ws=workspace())
 
 
 @pytest.mark.slow
@@ -116,9 +118,10 @@ def test_layer_sweep():
             check_act(t["dy"], fp8.BOTH)
             check_weight(t["w"])
             rows = pick_rows(syn.TOKENS, SWEEP_SAMPLE, seed)
-            check_fprop(t["x"], t["w"], rows, f"layer {seed} {name} fprop")
-            check_dgrad(t["dy"], t["w"], rows, f"layer {seed} {name} dgrad")
-            check_wgrad(t["dy"], t["x"], pick_rows(n, SWEEP_SAMPLE, seed + 1), f"layer {seed} {name} wgrad")
+            ws = workspace() if seed % 2 == 0 else None      # both schedules across the sweep
+            check_fprop(t["x"], t["w"], rows, f"layer {seed} {name} fprop", ws=ws)
+            check_dgrad(t["dy"], t["w"], rows, f"layer {seed} {name} dgrad", ws=ws)
+            check_wgrad(t["dy"], t["x"], pick_rows(n, SWEEP_SAMPLE, seed + 1), f"layer {seed} {name} wgrad", ws=ws)
 
 
 def test_heavy_tail_quantize_sweep():

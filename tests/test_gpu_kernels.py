@@ -12,7 +12,7 @@ import oracle
 from blockwise_fp8_pretraining_b200 import synthetic as syn
 
 from _parity import (assert_bits_equal, assert_within_bound, check_act, check_dgrad, check_fprop,
-                     check_wgrad, check_weight, dev, pick_rows)
+                     check_wgrad, check_weight, dev, pick_rows, workspace)
 
 pytestmark = pytest.mark.gpu
 
@@ -127,45 +127,59 @@ GEMM_SHAPES = [
 ]
 
 
+# With a workspace, shapes whose last wave of 256 x 256 tiles would leave
+# pairs idle run the split schedule (slab ranges per pair, partial sums
+# added by the pair holding each tile's first slab); without one, whole
+# tiles.  Both must meet the bound.
+SPLIT = [False, True]
+
+
+@pytest.mark.parametrize("split", SPLIT)
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-def test_fprop_small(M, N, K):
+def test_fprop_small(M, N, K, split):
     g = syn.generator(M + N + K)
     x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
     w = syn.normal_bf16((N, K), 0.02, g)
     rows = None if M <= 384 else pick_rows(M, 96, M)
-    check_fprop(x, w, rows, output_rounding=True)
+    check_fprop(x, w, rows, output_rounding=True, ws=workspace() if split else None)
 
 
+@pytest.mark.parametrize("split", SPLIT)
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-def test_dgrad_small(M, N, K):
+def test_dgrad_small(M, N, K, split):
     # dX [M, K] = dY [M, N] W [N, K]
     g = syn.generator(M * 7 + N + K)
     dy = syn.normal_bf16((M, N), 1e-3, g)
     w = syn.normal_bf16((N, K), 0.02, g)
     rows = None if M <= 384 else pick_rows(M, 96, M)
-    check_dgrad(dy, w, rows, output_rounding=True)
+    check_dgrad(dy, w, rows, output_rounding=True, ws=workspace() if split else None)
 
 
+@pytest.mark.parametrize("split", SPLIT)
 @pytest.mark.parametrize("N,K,M", [(128, 128, 128), (384, 256, 256), (256, 640, 384),
-                                   (1280, 2304, 256), (2560, 4096, 128)])
-def test_wgrad_small(N, K, M):
+                                   (1280, 2304, 256), (2560, 4096, 128), (2048, 2048, 1152)])
+def test_wgrad_small(N, K, M, split):
     g = syn.generator(N * 5 + K + M)
     dy = syn.normal_bf16((M, N), 1e-3, g)
     x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
     rows = None if N <= 384 else pick_rows(N, 96, N)
-    check_wgrad(dy, x, rows, output_rounding=True)
+    check_wgrad(dy, x, rows, output_rounding=True, ws=workspace() if split else None)
 
 
-def test_longest_contraction():
+@pytest.mark.parametrize("split", SPLIT)
+def test_longest_contraction(split):
     """The longest contraction the fprop/dgrad entry points accept (256 slabs
-    of 128), and a wgrad over as many tokens: every output element."""
+    of 128), and a wgrad over as many tokens: every output element.  With the
+    split schedule each of these single-tile GEMMs is cut into one slab range
+    per CTA pair, and one pair adds all the others' partial sums."""
     K = fp8.MAX_CONTRACTION_FPROP
     g = syn.generator(31)
-    check_fprop(syn.activation_bf16(256, K, K // 100, 30.0, g), syn.normal_bf16((256, K), 0.02, g))
+    ws = workspace() if split else None
+    check_fprop(syn.activation_bf16(256, K, K // 100, 30.0, g), syn.normal_bf16((256, K), 0.02, g), ws=ws)
     # dX [128, 256] = dY [128, K] W [K, 256]: the contraction runs over K
-    check_dgrad(syn.normal_bf16((128, K), 1e-3, g), syn.normal_bf16((K, 256), 0.02, g))
+    check_dgrad(syn.normal_bf16((128, K), 1e-3, g), syn.normal_bf16((K, 256), 0.02, g), ws=ws)
     # dW [256, 128] over K tokens
-    check_wgrad(syn.normal_bf16((K, 256), 1e-3, g), syn.activation_bf16(K, 128, 1, 30.0, g))
+    check_wgrad(syn.normal_bf16((K, 256), 1e-3, g), syn.activation_bf16(K, 128, 1, 30.0, g), ws=ws)
 
 
 def test_tiny_config_fprop_dgrad_wgrad_full():
@@ -217,7 +231,8 @@ def test_empty_inputs_are_noops():
 
 def test_outputs_do_not_depend_on_stream_or_repeat():
     """Same inputs on another stream and a second run give identical bits
-    (each output element is produced by one thread in a fixed order)."""
+    (each output element is produced by one thread in a fixed order, and
+    split tiles add their partial sums in a fixed order)."""
     c = syn.tiny(seed=3)
     d = dev()
     x, w = c["x"].to(d), c["w"].to(d)
@@ -230,6 +245,16 @@ def test_outputs_do_not_depend_on_stream_or_repeat():
     s.synchronize()
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+    # the split schedule: repeated runs, and a second workspace on another stream
+    ws2 = fp8.fp8_gemm_workspace()
+    y3 = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, workspace=workspace())
+    y4 = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, workspace=workspace())
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        y5 = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, workspace=ws2)
+    s.synchronize()
+    assert torch.equal(y3, y4) and torch.equal(y3, y5)
+    assert int(workspace().count_nonzero()) == 0 and int(ws2.count_nonzero()) == 0
 
 
 # --------------------------------------------------------------- time-outs
@@ -284,16 +309,16 @@ def test_gemm_writes_stay_inside_the_output(M, N, K):
     xq, sx, _, _ = fp8.fp8_quantize_act_1x128(x.to(d), fp8.ROWWISE)
     wq, sw, wqT = fp8.fp8_quantize_weight_128x128(w.to(d))
     buf, y = _guarded(M, N, torch.bfloat16, sentinel)
-    fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, y=y)
+    fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, y=y, workspace=workspace())
     dyq, sdy, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.BOTH)
     dbuf, dx = _guarded(M, K, torch.bfloat16, sentinel)
-    fp8.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=dx)
+    fp8.fp8_block_gemm_dgrad(dyq, sdy, wqT, sw, dx=dx, workspace=workspace())
     _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
     wbuf, dw = _guarded(N, K, torch.bfloat16, sentinel)
-    fp8.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=dw)
+    fp8.fp8_block_gemm_wgrad(dyqT, sdyT, xqT, sxT, dw=dw, workspace=workspace())
     fbuf, dwf = _guarded(N, K, torch.float32, 0x7FC0A5A5)
     dwf.zero_()
-    fp8.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dwf)
+    fp8.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dwf, workspace=workspace())
     torch.cuda.synchronize()
     _assert_guards(buf, M, sentinel, "fprop")
     _assert_guards(dbuf, M, sentinel, "dgrad")
@@ -323,7 +348,7 @@ def _accumulate(N, K, M, micro_batches, seed, rows=None):
         x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
         _, _, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.COLWISE)
         _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
-        fp8.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw)
+        fp8.fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, workspace=workspace() if b % 2 else None)
         dyqT_o, sdyT_o = oracle.quantize_act_colwise(syn.bf16_bits(dy))
         xqT_o, sxT_o = oracle.quantize_act_colwise(syn.bf16_bits(x))
         new, bound = oracle.gemm_wgrad_accum(dyqT_o, sdyT_o, xqT_o, sxT_o, running)
