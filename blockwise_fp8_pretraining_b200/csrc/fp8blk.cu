@@ -215,20 +215,23 @@ fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t*
 }
 
 // Workspace of the split schedule for `pairs` CTA pairs: FP32 partial sums
-// [pairs][2][EPI_WARPS][128][32], then one flag per pair, CTA and warp.
+// [pairs][2][EPI_WARPS][32][32][4], then one flag per pair, CTA, warp and lane.
 constexpr size_t kPartialFloatsPerPair = size_t(2) * gemm::EPI_WARPS * 128 * 32;
 inline size_t gemm_workspace_bytes(int pairs) {
     const size_t partial = size_t(pairs) * kPartialFloatsPerPair * sizeof(float);
-    const size_t flags = size_t(pairs) * 2 * gemm::EPI_WARPS * sizeof(int);
+    const size_t flags = size_t(pairs) * 2 * gemm::EPI_WARPS * 32 * sizeof(int);
     return (partial + flags + 255) / 256 * 256;
 }
 
 // Whole tiles round-robin for all waves but the last two when the last wave
-// would leave more than 5% of the pairs idle; those tiles are then cut into
-// ranges of slabs of equal length, one per pair.
-inline int dp_tiles_for(int64_t tiles, int pairs) {
+// would leave more than 5% of the pairs idle and a tile has at least 32 slabs;
+// those tiles are then cut into ranges of slabs of equal length, one per
+// pair.  (Measured on B200: with 16 slabs per tile the hand-over of partial
+// sums costs more than the idle pairs; from 32 slabs on the split gains.)
+constexpr int kMinSplitSlabs = 32;
+inline int dp_tiles_for(int64_t tiles, int pairs, int num_kb) {
     const int64_t waves = (tiles + pairs - 1) / pairs;
-    if (tiles >= waves * pairs * 95 / 100) return static_cast<int>(tiles);
+    if (num_kb < kMinSplitSlabs || tiles >= waves * pairs * 95 / 100) return static_cast<int>(tiles);
     const int64_t full = tiles / pairs;
     return static_cast<int>(full >= 1 ? (full - 1) * pairs : 0);
 }
@@ -282,8 +285,8 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Para
     p.dp_tiles = static_cast<int>(tiles);
     p.ws_partial = nullptr;
     p.ws_flags = nullptr;
-    if (workspace && workspace_bytes >= gemm_workspace_bytes(max_pairs) && p.K / gemm::BK > 1)
-        p.dp_tiles = dp_tiles_for(tiles, max_pairs);
+    if (workspace && workspace_bytes >= gemm_workspace_bytes(max_pairs))
+        p.dp_tiles = dp_tiles_for(tiles, max_pairs, p.K / gemm::BK);
     int grid_pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
     if (p.dp_tiles < tiles) {
         grid_pairs = max_pairs;
@@ -563,7 +566,7 @@ fp8_status fp8_selftest_gemm_schedule(int64_t M, int64_t N, int64_t K, int pairs
     p.tiles_m = static_cast<int>((M + 2 * gemm::BM - 1) / (2 * gemm::BM));
     p.tiles_n = static_cast<int>((N + gemm::BN - 1) / gemm::BN);
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-    p.dp_tiles = (split && p.K / gemm::BK > 1) ? dp_tiles_for(tiles, pairs) : static_cast<int>(tiles);
+    p.dp_tiles = split ? dp_tiles_for(tiles, pairs, p.K / gemm::BK) : static_cast<int>(tiles);
     const int npairs = p.dp_tiles < tiles ? pairs : static_cast<int>(tiles < pairs ? tiles : pairs);
     int64_t n = 0;
     for (int q = 0; q < npairs; ++q) {

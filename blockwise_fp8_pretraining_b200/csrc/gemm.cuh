@@ -134,8 +134,8 @@ struct Params {
     float* out_f32;         // main-gradient mode: the FP32 array [M, N] added to
     // Split schedule (see Schedule): tiles [0, dp_tiles) whole, the rest as
     // contiguous ranges of (tile, slab) units, partial sums through
-    // ws_partial [pairs][2][EPI_WARPS][128][32] f32 and ws_flags
-    // [pairs][2][EPI_WARPS] (zero between calls).  dp_tiles == total tiles
+    // ws_partial [pairs][2][EPI_WARPS][32][32 lanes][4] f32 and ws_flags
+    // [pairs][2][EPI_WARPS][32 lanes] (zero between calls).  dp_tiles == total tiles
     // means no split (the workspace is then unused and may be null).
     int dp_tiles;
     float* ws_partial;
@@ -415,6 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t tempty_leader = map_to_cta(bars.tempty, 0);
 
         float acc[128];
+        int* release_flag = nullptr;   // this lane's partial-sum flag, not yet released
         int it = 0;
         int ic = 0;        // scale chunks consumed
         bool ok = true;
@@ -497,6 +498,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
                 promote(ra, 64);
                 promote(rb, 96);
+                if (release_flag) {
+                    st_release_gpu(release_flag, 1);
+                    release_flag = nullptr;
+                }
                 if (j_in_chunk == SCHUNK - 1 || kb == sg.kb1 - 1) {
                     // last slab of this scale chunk: the slot may be refilled
                     __syncwarp();
@@ -508,14 +513,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
             if (sg.kb0 > 0) {
                 // A later part of a split tile: leave the partial sums to the
-                // pair that holds the tile's first slab.  Lane-fastest layout,
-                // so each store of the warp covers 128 contiguous bytes.
-                float* dst = p.ws_partial + ((static_cast<int64_t>(pair) * 2 + rank) * EPI_WARPS + ew) * (128 * 32);
+                // pair that holds the tile's first slab.  16-byte vectors,
+                // lane-fastest, so each store of the warp covers 512
+                // contiguous bytes; each lane then releases its own flag, which
+                // orders its stores before it (no fence for the whole warp).
+                const int64_t slot = (static_cast<int64_t>(pair) * 2 + rank) * EPI_WARPS + ew;
+                float4* dst = reinterpret_cast<float4*>(p.ws_partial) + slot * (32 * 32) + lane;
 #pragma unroll
-                for (int j = 0; j < 128; ++j) __stcg(dst + j * 32 + lane, acc[j]);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release_gpu(p.ws_flags + (pair * 2 + rank) * EPI_WARPS + ew, 1);
+                for (int j = 0; j < 32; ++j)
+                    __stcg(dst + j * 32, make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
+                // The flag is released one slab later (or when the pair's work
+                // ends): the release waits for the stores, which by then have
+                // landed, and the finalizing pair needs it only at the end of
+                // its own range.
+                release_flag = p.ws_flags + slot * 32 + lane;
                 continue;
             }
             if (sg.kb1 < sch.num_kb) {
@@ -525,7 +536,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const int64_t tile_end = static_cast<int64_t>(sg.tile + 1) * sch.num_kb - sch.sk_base;
                 for (int q = pair + 1; q < npairs && sch.range_begin(q) < tile_end; ++q) {
                     if (sch.range_begin(q) == sch.range_begin(q + 1)) continue;
-                    const int* flag = p.ws_flags + (q * 2 + rank) * EPI_WARPS + ew;
+                    const int64_t slot = (static_cast<int64_t>(q) * 2 + rank) * EPI_WARPS + ew;
+                    int* flag = p.ws_flags + slot * 32 + lane;
                     const uint64_t t0 = globaltimer_ns();
                     bool got = true;
                     while (ld_acquire_gpu(flag) == 0) {
@@ -542,11 +554,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         ok = false;
                         break;
                     }
-                    const float* src = p.ws_partial + ((static_cast<int64_t>(q) * 2 + rank) * EPI_WARPS + ew) * (128 * 32);
+                    const float4* src = reinterpret_cast<const float4*>(p.ws_partial) + slot * (32 * 32) + lane;
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) acc[j] += __ldcg(src + j * 32 + lane);
-                    __syncwarp();
-                    if (lane == 0) *const_cast<volatile int*>(flag) = 0;     // zero again for the next call
+                    for (int j = 0; j < 32; ++j) {
+                        const float4 v = __ldcg(src + j * 32);
+                        acc[4 * j] += v.x;
+                        acc[4 * j + 1] += v.y;
+                        acc[4 * j + 2] += v.z;
+                        acc[4 * j + 3] += v.w;
+                    }
+                    *const_cast<volatile int*>(flag) = 0;           // zero again for the next call
                 }
                 if (!ok) break;
             }
@@ -597,6 +614,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
+        if (release_flag) st_release_gpu(release_flag, 1);
         if (lane == 0) bulk_wait_group0();                 // output stores complete
     }
 

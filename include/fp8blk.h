@@ -92,8 +92,8 @@ enum {
  * workspace (workspace, workspace_bytes; NULL and 0 to go without).  With
  * one of at least fp8_gemm_workspace_bytes() bytes, a GEMM whose last wave
  * of 256x256 output tiles would leave more than 5% of the GPU's CTA pairs
- * idle cuts the tiles of its last two waves into equal ranges of 128-wide
- * contraction slabs, one range per pair; the pair holding a tile's first
+ * idle, and whose contraction has at least 32 slabs of 128, cuts the tiles
+ * of its last two waves into equal ranges of slabs, one range per pair; the pair holding a tile's first
  * slab adds the FP32 partial sums the other pairs leave in the workspace
  * (in a fixed order, so results are reproducible run to run) before its
  * epilogue.  Without a workspace every tile is computed whole by one pair.

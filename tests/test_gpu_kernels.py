@@ -166,6 +166,34 @@ def test_wgrad_small(N, K, M, split):
     check_wgrad(dy, x, rows, output_rounding=True, ws=workspace() if split else None)
 
 
+# Contractions of 32 slabs, where the split schedule applies: fewer tiles
+# than CTA pairs (every tile cut across pairs) and a partly idle last wave.
+SPLIT_SHAPES = [(256, 640, 4096), (1280, 2304, 4096), (4096, 2560, 4096)]
+
+
+@pytest.mark.parametrize("split", SPLIT)
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+def test_split_schedule_fprop_dgrad(M, N, K, split):
+    g = syn.generator(3 * M + N + K)
+    ws = workspace() if split else None
+    rows = None if M <= 256 else pick_rows(M, 96, M + 1)
+    check_fprop(syn.activation_bf16(M, K, K // 100, 30.0, g), syn.normal_bf16((N, K), 0.02, g), rows,
+                output_rounding=True, ws=ws)
+    # dX [M, N] = dY [M, K] W [K, N]: a K-deep contraction onto N columns
+    check_dgrad(syn.normal_bf16((M, K), 1e-3, g), syn.normal_bf16((K, N), 0.02, g), rows,
+                output_rounding=True, ws=ws)
+
+
+@pytest.mark.parametrize("split", SPLIT)
+@pytest.mark.parametrize("N,K,M", [(1280, 2304, 4096), (2560, 4096, 4096), (256, 256, 8192)])
+def test_split_schedule_wgrad(N, K, M, split):
+    g = syn.generator(N + 5 * K + M)
+    dy = syn.normal_bf16((M, N), 1e-3, g)
+    x = syn.activation_bf16(M, K, max(1, K // 100), 30.0, g)
+    rows = None if N <= 256 else pick_rows(N, 96, N + 2)
+    check_wgrad(dy, x, rows, output_rounding=True, ws=workspace() if split else None)
+
+
 @pytest.mark.parametrize("split", SPLIT)
 def test_longest_contraction(split):
     """The longest contraction the fprop/dgrad entry points accept (256 slabs
@@ -254,7 +282,13 @@ def test_outputs_do_not_depend_on_stream_or_repeat():
         y5 = fp8.fp8_block_gemm_fprop(xq, sx, wq, sw, workspace=ws2)
     s.synchronize()
     assert torch.equal(y3, y4) and torch.equal(y3, y5)
-    assert int(workspace().count_nonzero()) == 0 and int(ws2.count_nonzero()) == 0
+    # every flag is back to zero (the partial sums before them may remain):
+    # the workspace holds, per CTA pair, 262144 bytes of partial sums, then
+    # after all of those 2048 bytes of flags per pair
+    for w in (workspace(), ws2):
+        pairs = w.numel() // (262144 + 2048)
+        flags = w[pairs * 262144: pairs * (262144 + 2048)]
+        assert int(flags.count_nonzero()) == 0
 
 
 # --------------------------------------------------------------- time-outs
@@ -366,6 +400,12 @@ def _accumulate(N, K, M, micro_batches, seed, rows=None):
 @pytest.mark.parametrize("micro_batches", [2, 32])
 def test_wgrad_accumulates_in_fp32_over_micro_batches(micro_batches):
     _accumulate(384, 640, 256, micro_batches, seed=micro_batches)
+
+
+def test_wgrad_accumulates_with_the_split_schedule():
+    """A 4096-token wgrad (32 slabs, split across CTA pairs on odd micro-batches)
+    accumulated over 4 micro-batches."""
+    _accumulate(512, 768, 4096, 4, seed=77)
 
 
 @pytest.mark.slow

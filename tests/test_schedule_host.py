@@ -11,8 +11,8 @@ Invariants the kernel relies on:
   * the pair holding a tile's first slab, when the tile is split, adds the
     partial sums of exactly the pairs holding the tile's other slabs (its
     loop skips pairs whose split range is empty);
-  * without a workspace, or when the last wave is at least 95% full, tiles
-    are whole and assigned round-robin.
+  * without a workspace, with fewer than 32 slabs per tile, or when the last
+    wave is at least 95% full, tiles are whole and assigned round-robin.
 """
 import pytest
 
@@ -90,21 +90,23 @@ def test_schedule_invariants(lib, M, N, K, split):
             if kb0 == 0 and kb1 == nkb:
                 assert not holders
 
-    if not split or K == 128:
+    if not split or nkb < 32:
         assert all(kb0 == 0 and kb1 == nkb for _, _, kb0, kb1, _, _ in segs)
         for pair, tile, *_ in segs:
             assert tile % min(T, PAIRS) == pair
 
 
-@pytest.mark.parametrize("M,N,K", [(8192, 12288, 2048), (8192, 4096, 2048)])
+@pytest.mark.parametrize("M,N,K", [(8192, 12288, 2048), (8192, 4096, 2048), (8192, 2048, 2048),
+                                   (8192, 6144, 2048)])
 def test_full_last_waves_keep_whole_tiles(lib, M, N, K):
-    """At least 95% of the last wave busy: no split even with a workspace."""
+    """At least 95% of the last wave busy, or fewer than 32 slabs per tile:
+    no split even with a workspace."""
     segs = fp8.fp8_selftest_gemm_schedule(M, N, K, PAIRS, True)
     assert all(kb0 == 0 and kb1 == K // 128 for _, _, kb0, kb1, _, _ in segs)
 
 
-@pytest.mark.parametrize("M,N,K", [(8192, 2048, 2048), (2048, 2048, 8192), (12288, 2048, 8192),
-                                   (8192, 6144, 2048), (8192, 2048, 6144)])
+@pytest.mark.parametrize("M,N,K", [(8192, 2048, 4096), (2048, 2048, 8192), (12288, 2048, 8192),
+                                   (8192, 2048, 6144), (8192, 2048, 12288)])
 def test_partial_last_waves_are_balanced(lib, M, N, K):
     """With the split schedule every pair gets work, and the busiest pair
     has at most one slab more than the split share plus its whole tiles."""
