@@ -88,6 +88,8 @@ def parse():
                     help="--impl reference: oracle work of all warm-up and timed steps together")
     ap.add_argument("--graphs", type=int, default=8, help="distinct captured step graphs")
     ap.add_argument("--no-ceiling", action="store_true", help="skip the FP8 library ceiling measurement")
+    ap.add_argument("--no-split", action="store_true",
+                    help="GEMMs without a workspace: whole tiles only, no split schedule")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the per-launch timing of the fused SwiGLU producer and the FP32 main-grad wgrad")
     return ap.parse_args()
@@ -118,7 +120,7 @@ def step_gemm_flops(layers: int) -> float:
 class Sweep:
     """Device buffers and the launch list of one step."""
 
-    def __init__(self, layers: int, device, seed_base: int):
+    def __init__(self, layers: int, device, seed_base: int, no_split: bool = False):
         import torch
 
         from blockwise_fp8_pretraining_b200 import synthetic as syn
@@ -143,6 +145,8 @@ class Sweep:
 
         self.ws = fp8.fp8_gemm_workspace(device)
         self.ws_arg = (ctypes.c_void_p(self.ws.data_ptr()), ctypes.c_size_t(self.ws.numel()))
+        if no_split:
+            self.ws_arg = (ctypes.c_void_p(0), ctypes.c_size_t(0))
         self.layer = []
         for l in range(layers):
             gen = torch.Generator(device=device)
@@ -161,6 +165,14 @@ class Sweep:
     # A launch: (kind, c function name, argument builder taking the stream
     # handle and returning the ctypes argument tuple, flop, algorithmic bytes)
     def _launches_linear(self, per, sh, name, n, k, phase):
+        out = self._launches_linear_unlabeled(per, sh, name, n, k, phase)
+        labels = {"fp8_quantize_act_1x128": "quantize act", "fp8_quantize_weight_128x128": "quantize weight",
+                  "fp8_block_gemm_fprop": "fprop", "fp8_block_gemm_dgrad": "dgrad", "fp8_block_gemm_wgrad": "wgrad"}
+        return [(kind, fname, argf, flop, nbytes, f"{name} {labels[fname]}" +
+                 (" (dY)" if fname == "fp8_quantize_act_1x128" and phase == "bwd" else ""))
+                for kind, fname, argf, flop, nbytes in out]
+
+    def _launches_linear_unlabeled(self, per, sh, name, n, k, phase):
         T = TOKENS
         P = lambda t: ctypes.c_void_p(t.data_ptr())
         ws = self.ws_arg
@@ -219,7 +231,7 @@ def extra_launches(sweep):
         out.append(("swiglu_quant_fused", "fp8_swiglu_quantize_1x128",
                     lambda s, per=per: (P(gu["y"]), T, ffn, 3, P(dn["xq"]), P(dn["sx"]), P(per["xqT"]),
                                         P(per["sxT"]), s),
-                    0.0, T * ffn * (2 * 2 + 1 + 1 + 8 / 128)))
+                    0.0, T * ffn * (2 * 2 + 1 + 1 + 8 / 128), "fused SwiGLU producer"))
     if not hasattr(sweep, "main_grad"):
         sweep.main_grad = {name: torch.zeros((n, k), dtype=torch.float32, device=sweep.device)
                            for name, n, k in linear_shapes()}
@@ -230,13 +242,13 @@ def extra_launches(sweep):
                         lambda s, sh=sh, per=per, mg=mg, n=n, k=k: (P(sh["dyqT"]), P(sh["sdyT"]), P(per["xqT"]),
                                                                    P(per["sxT"]), P(mg), n, k, T,
                                                                    *sweep.ws_arg, s),
-                        2.0 * T * n * k, T * n + T * k + 2 * 4 * n * k))
+                        2.0 * T * n * k, T * n + T * k + 2 * 4 * n * k, f"{name} wgrad accumulate"))
     return out
 
 
 def run_launches(lib, launches, stream_handle, events=None):
     s = ctypes.c_void_p(stream_handle)
-    for i, (_, fname, argf, _, _) in enumerate(launches):
+    for i, (_, fname, argf, *_rest) in enumerate(launches):
         if events is not None:
             events[i].record()
         st = getattr(lib, fname)(*argf(s))
@@ -530,7 +542,7 @@ def summarize_kernels(launches, events_by_graph, pk, peak_kind):
     """Per kind: launches, total ms, share, and roofline numbers."""
     kinds = {}
     for events in events_by_graph:
-        for i, (kind, fname, _, flop, nbytes) in enumerate(launches):
+        for i, (kind, fname, _, flop, nbytes, *_label) in enumerate(launches):
             ms = events[i].elapsed_time(events[i + 1])
             d = kinds.setdefault(kind, {"launches": 0, "ms": 0.0, "flop": 0.0, "bytes": 0.0})
             d["launches"] += 1
@@ -544,6 +556,27 @@ def summarize_kernels(launches, events_by_graph, pk, peak_kind):
         d["tflops"] = d["flop"] / (d["ms"] * 1e-3) / 1e12 if d["flop"] else None
         d["gbs"] = d["bytes"] / (d["ms"] * 1e-3) / 1e9
     return kinds
+
+
+def summarize_labels(launches, events_by_graph):
+    """Mean device time per launch of each (linear, pass) of the step."""
+    acc = {}
+    for events in events_by_graph:
+        for i, (kind, fname, _, flop, nbytes, *label) in enumerate(launches):
+            if not label:
+                continue
+            d = acc.setdefault(label[0], {"n": 0, "ms": 0.0, "flop": flop, "bytes": nbytes})
+            d["n"] += 1
+            d["ms"] += events[i].elapsed_time(events[i + 1])
+    out = {}
+    for lab, d in acc.items():
+        us = 1e3 * d["ms"] / d["n"]
+        out[lab] = {"avg_us": round(us, 2)}
+        if d["flop"]:
+            out[lab]["tflops"] = round(d["flop"] / (us * 1e-6) / 1e12, 1)
+        else:
+            out[lab]["gbs"] = round(d["bytes"] / (us * 1e-6) / 1e9, 1)
+    return out
 
 
 def main_ours(args, rank, world, local_rank):
@@ -561,7 +594,7 @@ def main_ours(args, rank, world, local_rank):
     fp8.fp8_clear_error()
     pk, peak_kind = peaks()
 
-    sweep = Sweep(args.layers, device, seed_base=1000 * rank)
+    sweep = Sweep(args.layers, device, seed_base=1000 * rank, no_split=args.no_split)
     launches = sweep.launches()
     flop_step = step_gemm_flops(args.layers)
 
@@ -633,6 +666,7 @@ def main_ours(args, rank, world, local_rank):
         g.replay()
     torch.cuda.synchronize()
     kinds = summarize_kernels(launches, events_by_graph, pk, peak_kind)
+    by_label = summarize_labels(launches, events_by_graph)
     for g in prof_graphs:
         g.reset()
     prof_graphs.clear()
@@ -740,8 +774,9 @@ def main_ours(args, rank, world, local_rank):
                                    "micro-batch (2 x 4096)",
                        "tokens": TOKENS, "layers": args.layers, "gemm_tflop_per_step": flop_step / 1e12,
                        "launches_per_step": len(launches),
-                       "gemm_schedule": "split (slab ranges per CTA pair) where the last wave of 256x256 tiles "
-                                        "would leave >5% of pairs idle; whole tiles elsewhere",
+                       "gemm_schedule": ("whole 256x256 tiles (no workspace)" if args.no_split else
+                                         "split (slab ranges per CTA pair) where the last wave of 256x256 tiles "
+                                         "would leave >5% of pairs idle and K >= 32 slabs; whole tiles elsewhere"),
                        "l2": "no flush: 17.8 GB of distinct inputs per step >> 126 MB L2",
                        "parallelism": f"dp{world} replicas, no data-path collective"},
             "pct_of_fp8_dense_peak": 100.0 * value / FP8_DENSE_SPEC_TFLOPS,
@@ -754,6 +789,7 @@ def main_ours(args, rank, world, local_rank):
                                             roofline_fracs(d["tflops"], pk, peak_kind, ceiling).items()}}
                                if d["tflops"] else {})}
                         for k, d in kinds.items()},
+            "per_linear": by_label,
             "fp8_library_tflops": ceiling,
             "kernels_outside_step": extra,
             "roofline": roofline,
