@@ -16,6 +16,7 @@ from ._abi import (  # noqa: F401
     fp8_block_gemm_fprop,
     fp8_block_gemm_wgrad,
     fp8_block_gemm_wgrad_accum_f32,
+    fp8_block_gemm_wgrad_static_ws,
     fp8_cast_e4m3_scaled,
     fp8_clear_error,
     fp8_gemm_workspace,

@@ -64,6 +64,7 @@ def load() -> ctypes.CDLL:
         "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p, sz, p],
         "fp8_block_gemm_wgrad_accum_f32": [p, p, p, p, p, i64, i64, i64, p, sz, p],
         "fp8_gemm_workspace_bytes": [p],
+        "fp8_block_gemm_wgrad_static_ws": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_get_error": [],
         "fp8_clear_error": [],
         "fp8_set_wait_timeout_ns": [ctypes.c_uint64],
@@ -350,6 +351,27 @@ def fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, stream=None, worksp
     _check(lib.fp8_block_gemm_wgrad_accum_f32(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw),
                                               N, K, M, *_workspace(workspace), _stream(stream)),
            "fp8_block_gemm_wgrad_accum_f32")
+    return dw
+
+
+def fp8_block_gemm_wgrad_static_ws(dyqT, sdyT, xqT, sxT, dw=None, stream=None):
+    """dW = dY^T X (bf16) like fp8_block_gemm_wgrad, with the split
+    schedule's workspace inside the library (no device buffer passed), for
+    callers that cannot allocate one; calls must not overlap on the GPU."""
+    lib = load()
+    N, M = dyqT.shape
+    K = xqT.shape[0]
+    _want(dyqT, torch.uint8, (N, M), "dyqT")
+    _want(sdyT, torch.float32, (M // 128, N), "sdyT")
+    _want(xqT, torch.uint8, (K, M), "xqT")
+    _want(sxT, torch.float32, (M // 128, K), "sxT")
+    allocated = dw is None
+    dw = _out(dw, torch.bfloat16, (N, K), dyqT.device, "dw")
+    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("dw", dw)], stream)
+    _record(stream, [dw] if allocated else [])
+    _check(lib.fp8_block_gemm_wgrad_static_ws(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT), _ptr(dw), N, K, M,
+                                              _stream(stream)),
+           "fp8_block_gemm_wgrad_static_ws")
     return dw
 
 

@@ -323,6 +323,16 @@ bool dims_ok_gemm(int64_t M, int64_t N, int64_t K, bool m_positive) {
     return true;
 }
 
+// Scratch of fp8_block_gemm_wgrad_static_ws: the split schedule's workspace
+// as a file-scope device array, for callers that cannot allocate device
+// memory.  Every GPU that loads the library holds it until the process
+// exits; it starts zeroed (module load) and every call clears the flags it
+// needs zeroed.
+constexpr size_t kStaticWsBytes = size_t(24) << 20;     // 24 MiB: up to 94 CTA pairs
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+std::atomic<void*> g_static_ws_ptr[kMaxDevices];         // its device address, per device
+std::atomic<int> g_static_ws_pairs[kMaxDevices];         // resident GEMM CTA pairs, per device
+
 }  // namespace
 
 extern "C" {
@@ -466,6 +476,60 @@ fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t* dyqT, const float* sdyT
     return launch_gemm<gemm::kScaleOuter, gemm::kOutAccF32>(dyqT, xqT, dw_f32, wgrad_params(sdyT, sxT, N, K, M),
                                                             workspace, workspace_bytes,
                                                             static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_block_gemm_wgrad_static_ws(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
+                                          const float* sxT, void* dw_bf16, int64_t N, int64_t K, int64_t M,
+                                          void* stream) {
+    if (!dims_ok_gemm(N, K, M, true)) return FP8_ERR_SHAPE;
+    if (!dyqT || !sdyT || !xqT || !sxT || !dw_bf16) return FP8_ERR_NULL;
+    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(dw_bf16))
+        return FP8_ERR_ALIGN;
+    int dev = 0;
+    fp8_status st = current_device(&dev);
+    if (st != FP8_OK) return st;
+    void* ws = g_static_ws_ptr[dev].load(std::memory_order_acquire);
+    if (!ws) {
+        // Set-up, once per device, with that device current: the array's
+        // device address (the host-side name is only a stand-in for it) and
+        // the number of CTA pairs, which sizes the part of it in use.
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_ws);
+        if (e != cudaSuccess || !ptr) return cuda_fail("cudaGetSymbolAddress(static GEMM workspace)", e);
+        int sms = 0;
+        if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
+        e = cudaFuncSetAttribute(gemm::gemm_kernel<gemm::kScaleOuter, gemm::kOutBf16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+        cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
+        int pairs = 0;
+        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<gemm::kScaleOuter, gemm::kOutBf16>, &cfg);
+        if (e != cudaSuccess || pairs <= 0) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
+        g_static_ws_pairs[dev].store(pairs, std::memory_order_relaxed);
+        g_static_ws_ptr[dev].store(ptr, std::memory_order_release);
+        ws = ptr;
+    }
+    const int pairs = g_static_ws_pairs[dev].load(std::memory_order_relaxed);
+    const size_t need = gemm_workspace_bytes(pairs);
+    if (need > kStaticWsBytes) {
+        snprintf(g_detail, sizeof g_detail,
+                 "this GPU's GEMM workspace needs %zu bytes, more than the %zu-byte static one", need,
+                 kStaticWsBytes);
+        return FP8_ERR_SHAPE;
+    }
+    // The flags must be zero when a call starts; a call that timed out can
+    // leave some set, so they are cleared every time (a memset, not an
+    // allocation).
+    const size_t flags_off = size_t(pairs) * kPartialFloatsPerPair * sizeof(float);
+    const size_t flags_bytes = size_t(pairs) * 2 * gemm::EPI_WARPS * 32 * sizeof(int);
+    const cudaError_t e =
+        cudaMemsetAsync(static_cast<uint8_t*>(ws) + flags_off, 0, flags_bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(static GEMM workspace flags)", e);
+    return launch_gemm<gemm::kScaleOuter, gemm::kOutBf16>(dyqT, xqT, dw_bf16, wgrad_params(sdyT, sxT, N, K, M), ws,
+                                                          kStaticWsBytes, static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_gemm_workspace_bytes(size_t* bytes) {

@@ -255,6 +255,36 @@ fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t *dyqT, const float *sdyT
                                           void *workspace, size_t workspace_bytes,
                                           void *stream);
 
+/*
+ * wgrad for callers that cannot allocate device memory: the same GEMM as
+ * fp8_block_gemm_wgrad with the split schedule, whose workspace here is a
+ * fixed array inside the library instead of a buffer the caller passes.
+ * Some callers have no way to hand over a workspace: C code linked against
+ * this library without a GPU memory manager of its own, or programs whose
+ * framework allocator already holds (nearly) all device memory, or loops
+ * that must not pay for cudaMalloc and cudaFree, which can synchronize the
+ * device.  The pages have no counterpart to this entry point; it is a
+ * packaging convenience of this library.
+ *
+ *   dyqT, sdyT, xqT, sxT, dw_bf16, N, K, M - as fp8_block_gemm_wgrad; the
+ *   caller still owns and passes every input and output.
+ *
+ * Scratch: a file-scope device array of 24 MiB (enough for up to 94 CTA
+ * pairs; a 148-SM B200 uses 74), which every GPU that loads the library
+ * holds until the process exits.  A GPU that would need more returns
+ * FP8_ERR_SHAPE (fp8_last_cuda_error says how much).  The first call on a
+ * device looks up the array's device address and the GPU's CTA-pair count;
+ * make that first call before any stream capture.  Every call clears the
+ * array's flags with an asynchronous memset on `stream` and reuses the
+ * array's previous contents otherwise, so calls that may run at the same
+ * time on the GPU (different streams, or different host threads) race on
+ * it: order them on one stream.  Nothing is allocated or freed.
+ */
+fp8_status fp8_block_gemm_wgrad_static_ws(const uint8_t *dyqT, const float *sdyT,
+                                          const uint8_t *xqT, const float *sxT,
+                                          void *dw_bf16, int64_t N, int64_t K, int64_t M,
+                                          void *stream);
+
 /* Sticky per-device error word: FP8_OK, or the first FP8_ERR_TIMEOUT a
  * kernel recorded on the current device since the last clear.  Reading it
  * synchronizes the device. */
