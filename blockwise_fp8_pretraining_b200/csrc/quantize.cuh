@@ -283,22 +283,28 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
     }
     __syncthreads();
 
-    // Row pass: lanes l and l + 16 of a warp share row (l % 16) + 16 warp,
-    // one box (64 columns) each, so their maxima combine with one shuffle.
-    const int rrow = (lane & 15) + 16 * warp;
-    const int rbox = lane >> 4;        // row-pass box (columns 64 rbox ..)
-    const int p = t & 63;              // column-pass column pair
-    const int qq = t >> 6;             // column-pass row quarter
-    const int pbox = p >> 5;           // box holding columns 2p, 2p+1
-    const int pchunk = (p & 31) >> 2;  // their 16-byte chunk in the row
-    const int pbyte = (p & 3) * 4;     // their bytes in the chunk
-    // Column-pass byte offsets in a tile buffer of row qq * 32 + 8 i + u
-    // (u = 0..7) are coff[u] + 1024 i: the swizzle depends on the row only
-    // through r % 8, so eight offsets serve all 32 rows of the quarter.
+    // The two passes run side by side in two groups of four warps.
+    // Row group (warps 0-3): thread t owns row t of the tile and all 128 of
+    //   its columns (16 chunks of 8 bf16 in registers), so a 1x128 group needs
+    //   no exchange with other threads.
+    // Column group (warps 4-7): warp 4 + cw, lane l owns columns 2 l and
+    //   2 l + 1 of box (cw & 1) over rows 64 (cw >> 1) .. + 63, read as one
+    //   bf16 pair per row; a warp reads whole 128-byte rows of its box (no
+    //   bank conflicts).  The two row halves of a column combine their maxima
+    //   through shared memory and one named barrier of the column group.
+    //   Codes pack along the tokens directly (four rows per word).
+    const bool row_group = warp < 4;
+    const int cw = warp - 4;
+    const int cbox = cw & 1, chalf = cw >> 1;
+    const int cpair = cbox * 32 + lane;            // column pair within the tile
+    // Byte offset in a tile buffer of row 64 chalf + 8 i + u (u = 0..7) of
+    // the column thread's pair is coff[u] + 1024 i: the swizzle depends on
+    // the row only through r % 8.
     int coff[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u)
-        coff[u] = pbox * tile::BOX_BYTES + pbyte + qq * 32 * 128 + u * 128 + ((pchunk ^ u) << 4);
+        coff[u] = cbox * tile::BOX_BYTES + (64 * chalf + u) * 128 + (((lane >> 2) ^ u) << 4) + (lane & 3) * 4;
+    uint32_t* colx = reinterpret_cast<uint32_t*>(smem + L::OFF_COLS);   // [2 halves][64 pairs] partial maxima
 
     int i = 0;
     for (int64_t tl = blockIdx.x; tl < total; tl += gridDim.x, ++i) {
@@ -322,132 +328,123 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
             __syncthreads();
         }
 
-        // ---- row pass
-        const uint8_t* myrow = tin + rbox * tile::BOX_BYTES;
-        uint4 v[8];
+        // In weight mode both groups need the block's scale: the row group's
+        // warp maxima meet at named barrier 2 (all 256 threads; each group
+        // reaches it from its own branch).
+        if (row_group) {
+            // ---- row pass: codes of the thread's row into the row-layout staging
+            uint4 v[16];                 // the row: chunk k of box k / 8 at chunk k % 8
+            float sc = 0.0f;
+            if (want_rows || MODE == kTileWeight) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const uint4*>(myrow + tile::sw128(rrow, k));
-        // pairwise tree over the 8 chunk maxima (short dependency chains)
-        float a = fmaxf(fmaxf(fmaxf(amax8_packed(v[0]), amax8_packed(v[1])),
-                              fmaxf(amax8_packed(v[2]), amax8_packed(v[3]))),
-                        fmaxf(fmaxf(amax8_packed(v[4]), amax8_packed(v[5])),
-                              fmaxf(amax8_packed(v[6]), amax8_packed(v[7]))));
-        float block_scale = 0.0f;
-        if (MODE == kTileWeight) {
+                for (int k = 0; k < 16; ++k)
+                    v[k] = *reinterpret_cast<const uint4*>(tin + (k >> 3) * tile::BOX_BYTES + t * 128 +
+                                                           (((k & 7) ^ (t & 7)) << 4));
+                float m[4];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            if (lane == 0) red[warp] = a;
-            __syncthreads();
-            a = red[0];
+                for (int q = 0; q < 4; ++q)
+                    m[q] = fmaxf(fmaxf(amax8_packed(v[4 * q]), amax8_packed(v[4 * q + 1])),
+                                 fmaxf(amax8_packed(v[4 * q + 2]), amax8_packed(v[4 * q + 3])));
+                float a = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+                if (MODE == kTileWeight) {
 #pragma unroll
-            for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w]);
-            block_scale = group_scale(a);
-            if (t == 0) s_col[tr * tiles_c + tc] = block_scale;
-            __syncthreads();                            // red[] read before reuse below
-        } else if (want_rows) {
-            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
-        }
-        if (want_rows) {
-            const float sc = (MODE == kTileWeight) ? block_scale : group_scale(a);
-            if (MODE != kTileWeight && rbox == 0) s_row[tc * rows + r0 + rrow] = sc;
-            uint8_t* orow = smem + L::OFF_ROW;
-            const Quotient q(sc);
-            uint32_t out[16];
-            if (q.fast) {
-                const QuotientPair qp(q, q);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    out[2 * k] = qp.codes(v[k].x) | (qp.codes(v[k].y) << 16);
-                    out[2 * k + 1] = qp.codes(v[k].z) | (qp.codes(v[k].w) << 16);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    out[2 * k] = codes_pair_general(v[k].x, q, q) | (codes_pair_general(v[k].y, q, q) << 16);
-                    out[2 * k + 1] = codes_pair_general(v[k].z, q, q) | (codes_pair_general(v[k].w, q, q) << 16);
+                    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+                    if (lane == 0) red[warp] = a;
+                    named_bar_sync(2, tile::THREADS);
+                    sc = group_scale(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])));
+                    if (t == 0) s_col[tr * tiles_c + tc] = sc;
+                } else {
+                    sc = group_scale(a);
+                    s_row[tc * rows + r0 + t] = sc;
                 }
             }
+            if (want_rows) {
+                uint8_t* orow = smem + L::OFF_ROW + t * 128;
+                const Quotient q(sc);
+                if (q.fast) {
+                    const QuotientPair qp(q, q);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                *reinterpret_cast<uint4*>(orow + tile::sw128(rrow, 4 * rbox + k)) =
-                    make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
-        }
-
-        // ---- column pass
-        if (want_cols) {
-            // four independent running maxima, then combined
-            __nv_bfloat162 mq[4];
+                    for (int j = 0; j < 8; ++j) {       // output chunk j: input chunks 2j, 2j+1
+                        const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];
+                        const uint4 o = make_uint4(qp.codes(x0.x) | (qp.codes(x0.y) << 16),
+                                                   qp.codes(x0.z) | (qp.codes(x0.w) << 16),
+                                                   qp.codes(x1.x) | (qp.codes(x1.y) << 16),
+                                                   qp.codes(x1.z) | (qp.codes(x1.w) << 16));
+                        *reinterpret_cast<uint4*>(orow + ((j ^ (t & 7)) << 4)) = o;
+                    }
+                } else {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) mq[u] = __float2bfloat162_rn(0.0f);
-#pragma unroll
-            for (int rr = 0; rr < 32; ++rr) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(tin + coff[rr & 7] + (rr >> 3) * 1024);
-                mq[rr & 3] = __hmax2(mq[rr & 3], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
-            }
-            const __nv_bfloat162 m2 = __hmax2(__hmax2(mq[0], mq[1]), __hmax2(mq[2], mq[3]));
-            float s0 = block_scale, s1 = block_scale, rc0, rc1;
-            if (MODE != kTileWeight) {
-                const uint32_t mu = *reinterpret_cast<const uint32_t*>(&m2);
-                // (red[] and col_s[] were last read before the previous
-                // tile's closing barrier)
-                red[qq * kGroup + 2 * p] = __uint_as_float(mu << 16);
-                red[qq * kGroup + 2 * p + 1] = __uint_as_float(mu & 0xFFFF0000u);
-                __syncthreads();
-                // one thread per column finishes its scale and reciprocal
-                float* col_s = reinterpret_cast<float*>(smem + L::OFF_COLS);
-                if (t < kGroup) {
-                    const float am = fmaxf(fmaxf(red[t], red[kGroup + t]),
-                                           fmaxf(red[2 * kGroup + t], red[3 * kGroup + t]));
-                    const float sc = group_scale(am);
-                    col_s[t] = sc;
-                    col_s[kGroup + t] = Quotient(sc).r;
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];
+                        const uint4 o = make_uint4(
+                            codes_pair_general(x0.x, q, q) | (codes_pair_general(x0.y, q, q) << 16),
+                            codes_pair_general(x0.z, q, q) | (codes_pair_general(x0.w, q, q) << 16),
+                            codes_pair_general(x1.x, q, q) | (codes_pair_general(x1.y, q, q) << 16),
+                            codes_pair_general(x1.z, q, q) | (codes_pair_general(x1.w, q, q) << 16));
+                        *reinterpret_cast<uint4*>(orow + ((j ^ (t & 7)) << 4)) = o;
+                    }
                 }
-                __syncthreads();
-                s0 = col_s[2 * p];
-                s1 = col_s[2 * p + 1];
-                rc0 = col_s[kGroup + 2 * p];
-                rc1 = col_s[kGroup + 2 * p + 1];
-                if (qq == 0)
-                    *reinterpret_cast<float2*>(s_col + tr * cols + c0 + 2 * p) = make_float2(s0, s1);
-            } else {
-                const Quotient qb(block_scale);
-                rc0 = rc1 = qb.r;
             }
-            const Quotient q0(s0, rc0), q1(s1, rc1);
-            const bool fast = q0.fast && q1.fast;
-            const QuotientPair qp(s0, rc0, s1, rc1);
-            uint8_t* ocol = smem + L::OFF_COL;
-            // Codes of rows 4j .. 4j+3 of 16-token chunk 2qq + h for both
-            // columns, gathered into one word per column (row 4j lowest).
-            auto gather16 = [&](auto&& code_of, int h, uint32_t (&b0)[4], uint32_t (&b1)[4]) {
+        } else {
+            // ---- column pass: codes of the two columns along the tokens
+            float s0 = 0.0f, s1 = 0.0f;
+            if (MODE == kTileWeight) {
+                named_bar_sync(2, tile::THREADS);
+                s0 = s1 = group_scale(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])));
+            }
+            uint32_t w[64];              // the pair's two values of row 64 chalf + rr
+            if (want_cols) {
+#pragma unroll
+                for (int rr = 0; rr < 64; ++rr)
+                    w[rr] = *reinterpret_cast<const uint32_t*>(tin + coff[rr & 7] + (rr >> 3) * 1024);
+            }
+            if (MODE != kTileWeight && want_cols) {
+                __nv_bfloat162 mq[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mq[u] = __float2bfloat162_rn(0.0f);
+#pragma unroll
+                for (int rr = 0; rr < 64; ++rr)
+                    mq[rr & 3] = __hmax2(mq[rr & 3], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[rr])));
+                const __nv_bfloat162 m2 = __hmax2(__hmax2(mq[0], mq[1]), __hmax2(mq[2], mq[3]));
+                colx[chalf * 64 + cpair] = *reinterpret_cast<const uint32_t*>(&m2);
+                named_bar_sync(1, 128);             // the other row half's maxima are in
+                const uint32_t other = colx[(chalf ^ 1) * 64 + cpair];
+                const __nv_bfloat162 mm = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&other));
+                const uint32_t mu = *reinterpret_cast<const uint32_t*>(&mm);
+                s0 = group_scale(__uint_as_float(mu << 16));
+                s1 = group_scale(__uint_as_float(mu & 0xFFFF0000u));
+                if (chalf == 0) *reinterpret_cast<float2*>(s_col + tr * cols + c0 + 2 * cpair) = make_float2(s0, s1);
+            }
+            if (want_cols) {
+                const Quotient q0(s0), q1(s1);
+                const bool fast = q0.fast && q1.fast;
+                const QuotientPair qa(q0, q0), qb(q1, q1);
+                uint8_t* ocol = smem + L::OFF_COL;
+                const int ca = 2 * cpair, cb2 = 2 * cpair + 1;   // the two columns = rows of the transposed tile
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint32_t c[4];                      // codes (col 2p low byte, 2p+1 high byte)
+                    // words 4j .. 4j+3 of each column: rows 16 j + 4 k .. + 3, first row lowest
+                    uint32_t oa[4], ob[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int rl = h * 16 + 4 * j + u;     // row within the quarter
-                        const uint32_t w = *reinterpret_cast<const uint32_t*>(tin + coff[rl & 7] + (rl >> 3) * 1024);
-                        c[u] = code_of(w);
+                    for (int k = 0; k < 4; ++k) {
+                        const int r = 16 * j + 4 * k;
+                        const uint32_t w0 = w[r], w1 = w[r + 1], w2 = w[r + 2], w3 = w[r + 3];
+                        const uint32_t la = (w0 & 0xFFFFu) | (w1 << 16), lb = (w2 & 0xFFFFu) | (w3 << 16);
+                        const uint32_t ha = (w0 >> 16) | (w1 & 0xFFFF0000u), hb = (w2 >> 16) | (w3 & 0xFFFF0000u);
+                        if (fast) {
+                            oa[k] = qa.codes(la) | (qa.codes(lb) << 16);
+                            ob[k] = qb.codes(ha) | (qb.codes(hb) << 16);
+                        } else {
+                            oa[k] = codes_pair_general(la, q0, q0) | (codes_pair_general(lb, q0, q0) << 16);
+                            ob[k] = codes_pair_general(ha, q1, q1) | (codes_pair_general(hb, q1, q1) << 16);
+                        }
                     }
-                    const uint32_t lo01 = __byte_perm(c[0], c[1], 0x0040);  // c0.b0, c1.b0
-                    const uint32_t lo23 = __byte_perm(c[2], c[3], 0x0040);
-                    const uint32_t hi01 = __byte_perm(c[0], c[1], 0x0051);  // c0.b1, c1.b1
-                    const uint32_t hi23 = __byte_perm(c[2], c[3], 0x0051);
-                    b0[j] = __byte_perm(lo01, lo23, 0x5410);
-                    b1[j] = __byte_perm(hi01, hi23, 0x5410);
+                    const int chunk = 4 * chalf + j;
+                    *reinterpret_cast<uint4*>(ocol + ca * 128 + ((chunk ^ (ca & 7)) << 4)) =
+                        make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                    *reinterpret_cast<uint4*>(ocol + cb2 * 128 + ((chunk ^ (cb2 & 7)) << 4)) =
+                        make_uint4(ob[0], ob[1], ob[2], ob[3]);
                 }
-            };
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {               // 16-token chunks 2qq + h
-                uint32_t b0[4], b1[4];
-                if (fast)
-                    gather16([&](uint32_t w) { return qp.codes(w); }, h, b0, b1);
-                else
-                    gather16([&](uint32_t w) { return codes_pair_general(w, q0, q1); }, h, b0, b1);
-                const int chunk = 2 * qq + h;
-                const int c_a = 2 * p, c_b = 2 * p + 1;
-                *reinterpret_cast<uint4*>(ocol + tile::sw128(c_a, chunk)) = make_uint4(b0[0], b0[1], b0[2], b0[3]);
-                *reinterpret_cast<uint4*>(ocol + tile::sw128(c_b, chunk)) = make_uint4(b1[0], b1[1], b1[2], b1[3]);
             }
         }
 

@@ -10,14 +10,16 @@
 // the unfused H, so both roundings have to be the correctly rounded ones.
 //
 // silu(g) for a bfloat16 g is rounded once, correctly, to bfloat16:
-//   * 2^-20 <= |g| <= 80: FP32 evaluation g / (1 + expf(-g)) with the fast
-//     division __fdividef.  Its relative error is below 1.2 * 2^-21 (expf
-//     and __fdividef each within 2 units in the last place, one rounding of
-//     1 + e), while 32 float32 units in the last place at the result are at
-//     least 2^-19 of it.  So when the FP32 value lies more than
-//     32 float32 units from every bfloat16 rounding midpoint, it rounds like
-//     the exact value.  Otherwise (about one input in ten thousand) the
-//     element is evaluated in FP64.
+//   * 2^-20 <= |g| <= 80: FP32 evaluation g / (1 + e) with e = __expf(-g)
+//     and the fast division __fdividef.  __expf is within 2 + 1.173 |g|
+//     units in the last place (CUDA's documented bound for the intrinsic),
+//     __fdividef within 2, and 1 + e rounds once, so the quotient is within
+//     (5 + 1.173 |g|) * 2^-23 of silu(g), relative; a float32 unit in the
+//     last place at the result is at least 2^-24 of it, so the error is
+//     below 2 (5 + 1.173 |g|) < 12 + 3 |g| units.  When the FP32 value lies
+//     further than that (plus a margin of 8) from every bfloat16 rounding
+//     midpoint, it rounds like the exact value.  Otherwise (a fraction of a
+//     percent of inputs) the element is evaluated in FP64.
 //   * |g| < 2^-30: silu(g) = g/2 + g^2/4 + O(g^4).  g/2 is exact, and the
 //     positive g^2/4 term, far below a float32 unit at g/2, only decides
 //     the rounding when g/2 is a bfloat16 midpoint: the result is g/2 nudged
@@ -71,9 +73,11 @@ __device__ __noinline__ uint32_t silu_bf16_slow(float g) {
 __device__ __forceinline__ uint32_t silu_bf16(float g) {
     const float ag = fabsf(g);
     if (ag >= 0x1p-20f && ag <= 80.0f) {
-        const float q = __fdividef(g, 1.0f + expf(-g));
+        const float q = __fdividef(g, 1.0f + __expf(-g));
+        // units in the last place: 23 + 3 floor|g| >= 12 + 3|g| + 8
+        const int32_t margin = 23 + 3 * static_cast<int32_t>(ag);
         const int32_t from_mid = static_cast<int32_t>(__float_as_uint(q) & 0xFFFFu) - 0x8000;
-        if (from_mid > 32 || from_mid < -32) return bf16_rne_bits(q);
+        if (from_mid > margin || from_mid < -margin) return bf16_rne_bits(q);
     }
     return silu_bf16_slow(g);
 }
