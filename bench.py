@@ -762,7 +762,7 @@ def main_ours(args, rank, world, local_rank):
             sq["input"] = "each layer's gate_up fprop output [8192, 12288] (gate | up), both layouts out"
         oa = extra.get("gemm_outer_accum_f32")
         if oa:
-            oa["note"] = "wgrad of every linear added into FP32 main gradients (TMA reduce-add epilogue)"
+            oa["note"] = "wgrad of every linear added into FP32 main gradients (vector-reduction epilogue)"
 
     # ---- measured FP8 library ceiling (outside every timed region)
     ceiling = None if args.no_ceiling else fp8_library_ceiling(device)
@@ -835,7 +835,9 @@ def main_ours(args, rank, world, local_rank):
                        "launches_per_step": len(launches),
                        "gemm_schedule": ("whole 256x256 tiles (no workspace)" if args.no_split else
                                          "split (slab ranges per CTA pair) where the last wave of 256x256 tiles "
-                                         "would leave >5% of pairs idle and K >= 32 slabs; whole tiles elsewhere"),
+                                         "would leave >5% of pairs idle, K >= 32 slabs and the work is at least "
+                                         f"{fp8.GEMM_SPLIT_MIN_WORK_DEFAULT} tile-slabs per pair; whole tiles "
+                                         "elsewhere"),
                        "l2": "no flush: 17.8 GB of distinct inputs per step >> 126 MB L2",
                        "parallelism": f"dp{world} replicas, no data-path collective"},
             "pct_of_fp8_dense_peak": 100.0 * value / FP8_DENSE_SPEC_TFLOPS,

@@ -9,6 +9,7 @@ the built library raises.
 from ._abi import (  # noqa: F401
     BOTH,
     COLWISE,
+    GEMM_SPLIT_MIN_WORK_DEFAULT,
     MAX_CONTRACTION_FPROP,
     ROWWISE,
     Fp8Error,
@@ -30,6 +31,7 @@ from ._abi import (  # noqa: F401
     fp8_selftest_silu_bf16,
     fp8_selftest_stall_next,
     fp8_selftest_wait_timeout,
+    fp8_set_gemm_split_min_work,
     fp8_set_wait_timeout_ns,
     fp8_status_string,
     fp8_swiglu_quantize_1x128,

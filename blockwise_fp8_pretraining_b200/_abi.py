@@ -18,6 +18,7 @@ from . import build as _build
 
 ROWWISE, COLWISE, BOTH = 1, 2, 3
 MAX_CONTRACTION_FPROP = 32768
+GEMM_SPLIT_MIN_WORK_DEFAULT = 160      # FP8_GEMM_SPLIT_MIN_WORK_DEFAULT
 
 _lib = None
 
@@ -68,6 +69,7 @@ def load() -> ctypes.CDLL:
         "fp8_get_error": [],
         "fp8_clear_error": [],
         "fp8_set_wait_timeout_ns": [ctypes.c_uint64],
+        "fp8_set_gemm_split_min_work": [ctypes.c_int64],
         "fp8_cast_e4m3_scaled": [p, ctypes.c_float, p, i64, p],
         "fp8_selftest_wait_timeout": [p],
         "fp8_selftest_stall_next": [i32],
@@ -385,6 +387,10 @@ def fp8_clear_error() -> None:
 
 def fp8_set_wait_timeout_ns(ns: int) -> None:
     _check(load().fp8_set_wait_timeout_ns(int(ns)), "fp8_set_wait_timeout_ns")
+
+
+def fp8_set_gemm_split_min_work(units_per_pair: int) -> None:
+    _check(load().fp8_set_gemm_split_min_work(int(units_per_pair)), "fp8_set_gemm_split_min_work")
 
 
 def fp8_status_string(status: int) -> str:

@@ -56,7 +56,7 @@ inline uint32_t take_stall(int bit) {
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_gemm_attr_done[kMaxDevices];
-std::atomic<int> g_gemm_pairs[kMaxDevices][4];   // co-resident CTA pairs per kernel variant
+std::atomic<int> g_gemm_pairs[kMaxDevices][8];   // co-resident CTA pairs per kernel variant
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
@@ -224,21 +224,56 @@ inline size_t gemm_workspace_bytes(int pairs) {
 }
 
 // Whole tiles round-robin for all waves but the last two when the last wave
-// would leave more than 5% of the pairs idle and a tile has at least 32 slabs;
+// would leave more than 5% of the pairs idle, a tile has at least 32 slabs
+// and each pair has at least g_split_min_units (tile, slab) units of work;
 // those tiles are then cut into ranges of slabs of equal length, one per
-// pair.  (Measured on B200: with 16 slabs per tile the hand-over of partial
-// sums costs more than the idle pairs; from 32 slabs on the split gains.)
+// pair.  (Measured on B200: handing partial sums over costs a few
+// microseconds per launch, more than the idle pairs cost with 16 slabs per
+// tile or with under about 150 units per pair.)
 constexpr int kMinSplitSlabs = 32;
+constexpr int64_t kDefaultSplitMinUnits = FP8_GEMM_SPLIT_MIN_WORK_DEFAULT;
+std::atomic<int64_t> g_split_min_units{kDefaultSplitMinUnits};
 inline int dp_tiles_for(int64_t tiles, int pairs, int num_kb) {
     const int64_t waves = (tiles + pairs - 1) / pairs;
-    if (num_kb < kMinSplitSlabs || tiles >= waves * pairs * 95 / 100) return static_cast<int>(tiles);
+    if (num_kb < kMinSplitSlabs || tiles >= waves * pairs * 95 / 100 ||
+        tiles * num_kb < g_split_min_units.load(std::memory_order_relaxed) * pairs)
+        return static_cast<int>(tiles);
     const int64_t full = tiles / pairs;
     return static_cast<int>(full >= 1 ? (full - 1) * pairs : 0);
 }
 
+// One-time set-up of a GEMM kernel variant on a device: its shared-memory
+// limit, and how many CTA pairs can be resident at once (the persistent grid
+// must not exceed it, or the last pairs would wait for a second wave).
+template <int SCALE, int OUT, bool SPLIT>
+fp8_status gemm_pairs(int dev, int sms, int* pairs_out) {
+    constexpr int variant = SCALE + 2 * OUT + 4 * (SPLIT ? 1 : 0);
+    const int flag = 1 << variant;
+    if ((g_gemm_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
+        cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE, OUT, SPLIT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             gemm::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+        cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
+        int pairs = 0;
+        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<SCALE, OUT, SPLIT>, &cfg);
+        if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
+        if (pairs <= 0) return cuda_fail("gemm kernel cannot be resident", cudaErrorInvalidConfiguration);
+        g_gemm_pairs[dev][variant].store(pairs, std::memory_order_relaxed);
+        g_gemm_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
+    }
+    *pairs_out = g_gemm_pairs[dev][variant].load(std::memory_order_relaxed);
+    return FP8_OK;
+}
+
 // Shared launcher of the GEMMs.  A: [M_out, Kc] codes, B: [N_out, Kc]
 // codes, both K-major; scales described by `p`; out: [M_out, N_out] BF16, or
-// FP32 added to in place (OUT == kOutAccF32).
+// FP32 added to in place (OUT == kOutAccF32).  Launches the split-schedule
+// variant of the kernel only when the schedule splits tiles: the plain
+// variant's promotion loop carries nothing for it.
 template <int SCALE, int OUT>
 fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Params p, void* workspace,
                        size_t workspace_bytes, cudaStream_t stream) {
@@ -246,28 +281,8 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Para
     fp8_status st = current_device(&dev);
     if (st != FP8_OK) return st;
     if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
-
-    constexpr int variant = SCALE + 2 * OUT;
-    const int flag = 1 << variant;
-    if ((g_gemm_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE, OUT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             gemm::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
-        // How many CTA pairs can be resident at once: the persistent grid
-        // must not exceed it, or the last pairs would wait for a second wave.
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-        cfg.blockDim = dim3(gemm::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
-        int pairs = 0;
-        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<SCALE, OUT>, &cfg);
-        if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
-        if (pairs <= 0) return cuda_fail("gemm kernel cannot be resident", cudaErrorInvalidConfiguration);
-        g_gemm_pairs[dev][variant].store(pairs, std::memory_order_relaxed);
-        g_gemm_attr_done[dev].fetch_or(flag, std::memory_order_relaxed);
-    }
-    const int max_pairs = g_gemm_pairs[dev][variant].load(std::memory_order_relaxed);
+    int max_pairs = 0, split_pairs = 0;
+    if ((st = gemm_pairs<SCALE, OUT, false>(dev, sms, &max_pairs)) != FP8_OK) return st;
 
     CUtensorMap ma, mb, mc;
     if ((st = make_operand_map(&ma, a, p.M, p.K, gemm::BM)) != FP8_OK) return st;
@@ -287,16 +302,24 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Para
     p.ws_flags = nullptr;
     if (workspace && workspace_bytes >= gemm_workspace_bytes(max_pairs))
         p.dp_tiles = dp_tiles_for(tiles, max_pairs, p.K / gemm::BK);
-    int grid_pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
     if (p.dp_tiles < tiles) {
-        grid_pairs = max_pairs;
+        // Same resources as the plain variant, so the same residency; a
+        // smaller answer would leave pairs whose partial sums never arrive.
+        if ((st = gemm_pairs<SCALE, OUT, true>(dev, sms, &split_pairs)) != FP8_OK) return st;
+        if (split_pairs < max_pairs) p.dp_tiles = static_cast<int>(tiles);
+    }
+    cudaError_t e;
+    if (p.dp_tiles < tiles) {
         p.ws_partial = static_cast<float*>(workspace);
         p.ws_flags = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
                                             size_t(max_pairs) * kPartialFloatsPerPair * sizeof(float));
+        e = launch_pdl(gemm::gemm_kernel<SCALE, OUT, true>, dim3(2 * max_pairs), dim3(gemm::THREADS),
+                       gemm::SMEM_BYTES, stream, ma, mb, mc, p);
+    } else {
+        const int grid_pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+        e = launch_pdl(gemm::gemm_kernel<SCALE, OUT, false>, dim3(2 * grid_pairs), dim3(gemm::THREADS),
+                       gemm::SMEM_BYTES, stream, ma, mb, mc, p);
     }
-    const int grid = 2 * grid_pairs;
-    const cudaError_t e = launch_pdl(gemm::gemm_kernel<SCALE, OUT>, dim3(grid), dim3(gemm::THREADS),
-                                     gemm::SMEM_BYTES, stream, ma, mb, mc, p);
     if (e != cudaSuccess) return cuda_fail("gemm launch", e);
     return last_launch_status("gemm launch");
 }
@@ -496,18 +519,9 @@ fp8_status fp8_block_gemm_wgrad_static_ws(const uint8_t* dyqT, const float* sdyT
         void* ptr = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_ws);
         if (e != cudaSuccess || !ptr) return cuda_fail("cudaGetSymbolAddress(static GEMM workspace)", e);
-        int sms = 0;
+        int sms = 0, pairs = 0;
         if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
-        e = cudaFuncSetAttribute(gemm::gemm_kernel<gemm::kScaleOuter, gemm::kOutBf16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-        cfg.blockDim = dim3(gemm::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
-        int pairs = 0;
-        e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<gemm::kScaleOuter, gemm::kOutBf16>, &cfg);
-        if (e != cudaSuccess || pairs <= 0) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
+        if ((st = gemm_pairs<gemm::kScaleOuter, gemm::kOutBf16, false>(dev, sms, &pairs)) != FP8_OK) return st;
         g_static_ws_pairs[dev].store(pairs, std::memory_order_relaxed);
         g_static_ws_ptr[dev].store(ptr, std::memory_order_release);
         ws = ptr;
@@ -537,19 +551,10 @@ fp8_status fp8_gemm_workspace_bytes(size_t* bytes) {
     int dev = 0;
     fp8_status st = current_device(&dev);
     if (st != FP8_OK) return st;
-    int pairs = 0;
     // Resident CTA pairs of the GEMM kernels (all variants share one shape).
-    cudaLaunchConfig_t cfg = {};
-    int sms = 0;
+    int sms = 0, pairs = 0;
     if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
-    cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<gemm::kScaleRowBlock, gemm::kOutBf16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemm)", e);
-    cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-    cfg.blockDim = dim3(gemm::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
-    e = cudaOccupancyMaxActiveClusters(&pairs, gemm::gemm_kernel<gemm::kScaleRowBlock, gemm::kOutBf16>, &cfg);
-    if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters(gemm)", e);
+    if ((st = gemm_pairs<gemm::kScaleRowBlock, gemm::kOutBf16, false>(dev, sms, &pairs)) != FP8_OK) return st;
     *bytes = gemm_workspace_bytes(pairs);
     return FP8_OK;
 }
@@ -573,6 +578,12 @@ fp8_status fp8_clear_error(void) {
 }
 
 const char* fp8_last_cuda_error(void) { return g_detail; }
+
+fp8_status fp8_set_gemm_split_min_work(int64_t units_per_pair) {
+    if (units_per_pair < 0) return FP8_ERR_SHAPE;
+    g_split_min_units.store(units_per_pair, std::memory_order_relaxed);
+    return FP8_OK;
+}
 
 fp8_status fp8_set_wait_timeout_ns(uint64_t ns) {
     g_wait_ns.store(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);
@@ -632,11 +643,14 @@ fp8_status fp8_selftest_gemm_schedule(int64_t M, int64_t N, int64_t K, int pairs
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     p.dp_tiles = split ? dp_tiles_for(tiles, pairs, p.K / gemm::BK) : static_cast<int>(tiles);
     const int npairs = p.dp_tiles < tiles ? pairs : static_cast<int>(tiles < pairs ? tiles : pairs);
+    const bool split_launch = p.dp_tiles < tiles;
+    const int num_kb = p.K / gemm::BK;
     int64_t n = 0;
     for (int q = 0; q < npairs; ++q) {
-        gemm::Schedule sch(p, q, npairs);
         gemm::Seg sg;
-        while (sch.next(sg)) {
+        for (int idx = 0; split_launch ? gemm::segment<true>(p, q, npairs, idx, sg)
+                                       : gemm::segment<false>(p, q, npairs, idx, sg);
+             ++idx) {
             if (n >= max_segs) return FP8_ERR_SHAPE;
             int32_t* row = segs + 5 * n;
             row[0] = q;
@@ -646,11 +660,13 @@ fp8_status fp8_selftest_gemm_schedule(int64_t M, int64_t N, int64_t K, int pairs
             // the pairs whose partial sums a finalizing segment adds: the
             // first and one past the last (equal when none)
             int32_t first = 0, last = 0;
-            if (sg.kb0 == 0 && sg.kb1 < sch.num_kb) {
-                const int64_t tile_end = static_cast<int64_t>(sg.tile + 1) * sch.num_kb - sch.sk_base;
+            if (sg.kb0 == 0 && sg.kb1 < num_kb) {
+                const int64_t tile_end =
+                    static_cast<int64_t>(sg.tile + 1) * num_kb - static_cast<int64_t>(p.dp_tiles) * num_kb;
                 first = q + 1;
                 last = q + 1;
-                for (int r = q + 1; r < npairs && sch.range_begin(r) < tile_end; ++r) last = r + 1;
+                for (int r = q + 1; r < npairs && gemm::split_range_begin(p, r, npairs) < tile_end; ++r)
+                    last = r + 1;
             }
             row[4] = (first << 16) | last;
             ++n;

@@ -155,37 +155,47 @@ struct Seg {
     int tile, kb0, kb1;
 };
 
-struct Schedule {
-    int num_kb, dp_tiles, npairs, next_dp;
-    int64_t u, u_end, sk_base, sk_units;
-    __host__ __device__ __forceinline__ Schedule(const Params& p, int pair, int npairs_)
-        : num_kb(p.K / BK), dp_tiles(p.dp_tiles), npairs(npairs_), next_dp(pair) {
-        const int total = p.tiles_m * p.tiles_n;
-        sk_base = static_cast<int64_t>(dp_tiles) * num_kb;
-        sk_units = static_cast<int64_t>(total - dp_tiles) * num_kb;
-        u = sk_base + range_begin(pair);
-        u_end = sk_base + range_begin(pair + 1);
+// First unit (relative to the split part, which starts at unit
+// dp_tiles * num_kb) of pair q's range.
+__host__ __device__ __forceinline__ int64_t split_range_begin(const Params& p, int q, int npairs) {
+    const int64_t units = static_cast<int64_t>(p.tiles_m * p.tiles_n - p.dp_tiles) * (p.K / BK);
+    return units * q / npairs;
+}
+
+// Segment `idx` of pair `pair`'s work, or false past the last one.  It is
+// computed from the launch parameters and idx alone: the roles carry only
+// the index from one segment to the next, so the schedule adds no live
+// registers to the promotion warps' slab loop (whose accumulators leave
+// almost none spare).  SPLIT == false is the plain round-robin of whole tiles.
+template <bool SPLIT>
+__host__ __device__ __forceinline__ bool segment(const Params& p, int pair, int npairs, int idx, Seg& sg) {
+    const int num_kb = p.K / BK;
+    if (!SPLIT) {
+        sg.tile = pair + idx * npairs;
+        sg.kb0 = 0;
+        sg.kb1 = num_kb;
+        return sg.tile < p.tiles_m * p.tiles_n;
     }
-    // First unit (relative to sk_base) of pair q's range.
-    __host__ __device__ __forceinline__ int64_t range_begin(int q) const { return sk_units * q / npairs; }
-    __host__ __device__ __forceinline__ bool next(Seg& sg) {
-        if (next_dp < dp_tiles) {
-            sg.tile = next_dp;
-            sg.kb0 = 0;
-            sg.kb1 = num_kb;
-            next_dp += npairs;
-            return true;
-        }
-        if (u >= u_end) return false;
-        sg.tile = static_cast<int>(u / num_kb);
-        sg.kb0 = static_cast<int>(u - static_cast<int64_t>(sg.tile) * num_kb);
-        const int64_t left = u_end - u;
-        const int64_t end = sg.kb0 + left;
-        sg.kb1 = static_cast<int>(end < num_kb ? end : num_kb);
-        u += sg.kb1 - sg.kb0;
+    const int n_dp = pair < p.dp_tiles ? (p.dp_tiles - 1 - pair) / npairs + 1 : 0;
+    if (idx < n_dp) {
+        sg.tile = pair + idx * npairs;
+        sg.kb0 = 0;
+        sg.kb1 = num_kb;
         return true;
     }
-};
+    const int64_t base = static_cast<int64_t>(p.dp_tiles) * num_kb;
+    const int64_t b = base + split_range_begin(p, pair, npairs);
+    const int64_t e = base + split_range_begin(p, pair + 1, npairs);
+    const int64_t j = idx - n_dp;
+    // the first segment starts where the range does, later ones at tile starts
+    const int64_t start = (j == 0) ? b : (b / num_kb + j) * num_kb;
+    if (start >= e) return false;
+    sg.tile = static_cast<int>(start / num_kb);
+    const int64_t tile_u = static_cast<int64_t>(sg.tile) * num_kb;
+    sg.kb0 = static_cast<int>(start - tile_u);
+    sg.kb1 = static_cast<int>(e - tile_u < num_kb ? e - tile_u : num_kb);
+    return true;
+}
 
 // Release / acquire flag accesses for the partial-sum hand-over between pairs.
 __device__ __forceinline__ void st_release_gpu(int* addr, int v) {
@@ -210,7 +220,7 @@ struct Bars {
 // tmA: A codes [M, K] (box 128 x 128), tmB: B codes [N, K] (box 128 x 128),
 // tmC: BF16 output [M, N], box 64 x 32, 128-byte swizzled (kOutBf16; in
 // main-gradient mode p.out_f32 is written instead).
-template <int SCALE, int OUT>
+template <int SCALE, int OUT, bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const Params p) {
@@ -275,9 +285,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const uint32_t full_leader = map_to_cta(bars.full, 0);
             int it = 0;    // slabs whose operand tiles were requested
             bool ok = true;
-            Schedule sch(p, pair, npairs);
             Seg sg;
-            while (ok && sch.next(sg)) {
+            for (int seg = 0; ok && segment<SPLIT>(p, pair, npairs, seg, sg); ++seg) {
                 const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
                 const int n0 = (sg.tile % p.tiles_n) * BN;
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
@@ -312,9 +321,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // bulk copy) and store them into the slot before lane 0 arrives.
         int ic = 0;    // scale chunks requested
         bool ok = true;
-        Schedule sch(p, pair, npairs);
         Seg sg;
-        while (ok && sch.next(sg)) {
+        for (int seg = 0; ok && segment<SPLIT>(p, pair, npairs, seg, sg); ++seg) {
             const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
             const int n0 = (sg.tile % p.tiles_n) * BN;
             const uint32_t sa_bytes = (m_own < p.M) ? BM * 4u : 0u;
@@ -367,10 +375,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int sel = (warp == 1) ? 0 : 1;
             int it = 0;
             bool ok = true;
-            Schedule sch(p, pair, npairs);
             Seg sg;
-            while (ok && sch.next(sg)) {
-                for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+            for (int seg = 0; ok && segment<SPLIT>(p, pair, npairs, seg, sg); ++seg) {
+                const int nslab = sg.kb1 - sg.kb0;
+                for (int j = 0; j < nslab; ++j, ++it) {
                     if ((it & 1) != sel) continue;
                     const int buf = it & 1;
                     if (!mbar_wait(bars.tempty_(buf), ((it >> 1) & 1) ^ 1, abort_flag, p.wait_ns, kErrTimeout,
@@ -415,22 +423,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t tempty_leader = map_to_cta(bars.tempty, 0);
 
         float acc[128];
-        int* release_flag = nullptr;   // this lane's partial-sum flag, not yet released
+        bool pending = false;   // split only: this lane's partial-sum flag is still to be released
         int it = 0;
         int ic = 0;        // scale chunks consumed
         bool ok = true;
-        Schedule sch(p, pair, npairs);
-        Seg sg;
-        while (ok && sch.next(sg)) {
-            const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
-            const int n0 = (sg.tile % p.tiles_n) * BN;
+        for (int seg = 0; ok; ++seg) {
+            Seg sg;
+            if (!segment<SPLIT>(p, pair, npairs, seg, sg)) break;
+            const int nslab = sg.kb1 - sg.kb0;
 #pragma unroll
             for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
 
-            for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+            for (int js = 0; js < nslab; ++js, ++it) {
                 const int buf = it & 1;
                 const int sl = ic % SSLOTS;
-                const int j_in_chunk = (kb - sg.kb0) % SCHUNK;
+                const int j_in_chunk = js % SCHUNK;
                 bool got = true;
                 if (j_in_chunk == 0)
                     got = mbar_wait(bars.sfull_(sl), (ic / SSLOTS) & 1, abort_flag, p.wait_ns, kErrTimeout);
@@ -498,11 +505,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
                 promote(ra, 64);
                 promote(rb, 96);
-                if (release_flag) {
-                    st_release_gpu(release_flag, 1);
-                    release_flag = nullptr;
+                if (SPLIT && pending) {
+                    st_release_gpu(p.ws_flags + ((pair * 2 + static_cast<int>(rank)) * EPI_WARPS + ew) * 32 + lane, 1);
+                    pending = false;
                 }
-                if (j_in_chunk == SCHUNK - 1 || kb == sg.kb1 - 1) {
+                if (j_in_chunk == SCHUNK - 1 || js == nslab - 1) {
                     // last slab of this scale chunk: the slot may be refilled
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bars.sempty_(sl));
@@ -510,68 +517,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
             if (!ok) break;
-
-            if (sg.kb0 > 0) {
-                // A later part of a split tile: leave the partial sums to the
-                // pair that holds the tile's first slab.  16-byte vectors,
-                // lane-fastest, so each store of the warp covers 512
-                // contiguous bytes; each lane then releases its own flag, which
-                // orders its stores before it (no fence for the whole warp).
-                const int64_t slot = (static_cast<int64_t>(pair) * 2 + rank) * EPI_WARPS + ew;
-                float4* dst = reinterpret_cast<float4*>(p.ws_partial) + slot * (32 * 32) + lane;
+            if (SPLIT) {
+                // The segment again, from its index alone (the opaque move
+                // keeps the compiler from carrying the first lookup's values
+                // across the slab loop).
+                asm volatile("" : "+r"(seg));
+                segment<true>(p, pair, npairs, seg, sg);
+                if (sg.kb0 > 0) {
+                    // A later part of a split tile: leave the partial sums to
+                    // the pair that holds the tile's first slab.  16-byte
+                    // vectors, lane-fastest, so each store of the warp covers
+                    // 512 contiguous bytes.  Each lane releases its own flag
+                    // one slab later (or when the pair's work ends): the
+                    // release orders the lane's stores before it, they have
+                    // landed by then, and the finalizing pair needs them only
+                    // at the end of its own range.
+                    const int64_t slot = (static_cast<int64_t>(pair) * 2 + rank) * EPI_WARPS + ew;
+                    float4* dst = reinterpret_cast<float4*>(p.ws_partial) + slot * (32 * 32) + lane;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    __stcg(dst + j * 32, make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
-                // The flag is released one slab later (or when the pair's work
-                // ends): the release waits for the stores, which by then have
-                // landed, and the finalizing pair needs it only at the end of
-                // its own range.
-                release_flag = p.ws_flags + slot * 32 + lane;
-                continue;
-            }
-            if (sg.kb1 < sch.num_kb) {
-                // The first part of a split tile: add the partial sums of the
-                // pairs holding the rest, in pair order, then the epilogue.
-                // (A pair with an empty range holds nothing.)
-                const int64_t tile_end = static_cast<int64_t>(sg.tile + 1) * sch.num_kb - sch.sk_base;
-                for (int q = pair + 1; q < npairs && sch.range_begin(q) < tile_end; ++q) {
-                    if (sch.range_begin(q) == sch.range_begin(q + 1)) continue;
-                    const int64_t slot = (static_cast<int64_t>(q) * 2 + rank) * EPI_WARPS + ew;
-                    int* flag = p.ws_flags + slot * 32 + lane;
-                    const uint64_t t0 = globaltimer_ns();
-                    bool got = true;
-                    while (ld_acquire_gpu(flag) == 0) {
-                        if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
-                            if (!*abort_flag) {
-                                record_error(kErrTimeout);
-                                *abort_flag = 1;
+                    for (int j = 0; j < 32; ++j)
+                        __stcg(dst + j * 32, make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
+                    pending = true;
+                    continue;
+                }
+                const int num_kb = p.K / BK;
+                if (sg.kb1 < num_kb) {
+                    // The first part of a split tile: add the partial sums of
+                    // the pairs holding the rest, in pair order, then the
+                    // epilogue.  (A pair with an empty range holds nothing.)
+                    const int64_t tile_end =
+                        static_cast<int64_t>(sg.tile + 1) * num_kb - static_cast<int64_t>(p.dp_tiles) * num_kb;
+                    for (int q = pair + 1; q < npairs && split_range_begin(p, q, npairs) < tile_end; ++q) {
+                        if (split_range_begin(p, q, npairs) == split_range_begin(p, q + 1, npairs)) continue;
+                        const int64_t slot = (static_cast<int64_t>(q) * 2 + rank) * EPI_WARPS + ew;
+                        int* flag = p.ws_flags + slot * 32 + lane;
+                        const uint64_t t0 = globaltimer_ns();
+                        bool got = true;
+                        while (ld_acquire_gpu(flag) == 0) {
+                            if (*abort_flag || globaltimer_ns() - t0 > p.wait_ns) {
+                                if (!*abort_flag) {
+                                    record_error(kErrTimeout);
+                                    *abort_flag = 1;
+                                }
+                                got = false;
+                                break;
                             }
-                            got = false;
+                        }
+                        if (!__all_sync(0xffffffffu, got)) {
+                            ok = false;
                             break;
                         }
-                    }
-                    if (!__all_sync(0xffffffffu, got)) {
-                        ok = false;
-                        break;
-                    }
-                    const float4* src = reinterpret_cast<const float4*>(p.ws_partial) + slot * (32 * 32) + lane;
+                        const float4* src = reinterpret_cast<const float4*>(p.ws_partial) + slot * (32 * 32) + lane;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float4 v = __ldcg(src + j * 32);
-                        acc[4 * j] += v.x;
-                        acc[4 * j + 1] += v.y;
-                        acc[4 * j + 2] += v.z;
-                        acc[4 * j + 3] += v.w;
+                        for (int j = 0; j < 32; ++j) {
+                            const float4 v = __ldcg(src + j * 32);
+                            acc[4 * j] += v.x;
+                            acc[4 * j + 1] += v.y;
+                            acc[4 * j + 2] += v.z;
+                            acc[4 * j + 3] += v.w;
+                        }
+                        *const_cast<volatile int*>(flag) = 0;       // zero again for the next call
                     }
-                    *const_cast<volatile int*>(flag) = 0;           // zero again for the next call
+                    if (!ok) break;
                 }
-                if (!ok) break;
             }
 
             // BF16 round-to-nearest-even into this warp's staging buffer (two
             // 32 x 64 boxes, 128-byte rows, 16-byte chunk j of row r at
             // position j ^ (r % 8)), then TMA stores of the two boxes.
-            const int col0 = n0 + half * 128;
+            const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
+            const int col0 = (sg.tile % p.tiles_n) * BN + half * 128;
             if (OUT == kOutAccF32 && col0 < p.N && m_own < p.M) {
                 // FP32 added to the array in memory straight from the
                 // registers: one vector reduction per 4 columns, so each
@@ -614,7 +629,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
-        if (release_flag) st_release_gpu(release_flag, 1);
+        if (SPLIT && pending)
+            st_release_gpu(p.ws_flags + ((pair * 2 + static_cast<int>(rank)) * EPI_WARPS + ew) * 32 + lane, 1);
         if (lane == 0) bulk_wait_group0();                 // output stores complete
     }
 

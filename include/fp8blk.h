@@ -92,12 +92,14 @@ enum {
  * workspace (workspace, workspace_bytes; NULL and 0 to go without).  With
  * one of at least fp8_gemm_workspace_bytes() bytes, a GEMM whose last wave
  * of 256x256 output tiles would leave more than 5% of the GPU's CTA pairs
- * idle, and whose contraction has at least 32 slabs of 128, cuts the tiles
- * of its last two waves into equal ranges of slabs, one range per pair; the pair holding a tile's first
- * slab adds the FP32 partial sums the other pairs leave in the workspace
- * (in a fixed order, so results are reproducible run to run) before its
- * epilogue.  Without a workspace every tile is computed whole by one pair.
- * Either way every output element satisfies the same error bound.
+ * idle, whose contraction has at least 32 slabs of 128, and whose work is
+ * at least fp8_set_gemm_split_min_work's threshold per pair, cuts the tiles
+ * of its last two waves into equal ranges of slabs, one range per pair; the
+ * pair holding a tile's first slab adds the FP32 partial sums the other
+ * pairs leave in the workspace (in a fixed order, so results are
+ * reproducible run to run) before its epilogue.  Without a workspace every
+ * tile is computed whole by one pair.  Either way every output element
+ * satisfies the same error bound.
  *
  * The workspace is owned by the caller, 16-byte aligned, and must hold
  * zeros before its first use (cudaMemset); every call that completes leaves
@@ -107,6 +109,20 @@ enum {
  * device (about 19 MB on a 148-SM B200).
  */
 fp8_status fp8_gemm_workspace_bytes(size_t *bytes);
+
+/*
+ * Least work per CTA pair, in units of one 256x256 tile times one slab of
+ * 128, for which a GEMM given a workspace uses the split schedule (default
+ * FP8_GEMM_SPLIT_MIN_WORK_DEFAULT).  Handing the partial sums over costs a few microseconds per launch,
+ * so on a B200 the split gains only on long GEMMs: with it the 8192-token
+ * gate_up wgrad (332 units per pair) ran 4% faster and the o_proj wgrad (55
+ * units per pair) 10% slower.  0 lets the split apply whenever the other two
+ * conditions hold.  Negative values return FP8_ERR_SHAPE.  Host-side
+ * setting, shared by all devices and threads; it takes effect for launches
+ * made after the call.
+ */
+#define FP8_GEMM_SPLIT_MIN_WORK_DEFAULT 160
+fp8_status fp8_set_gemm_split_min_work(int64_t units_per_pair);
 
 /*
  * Activation quantizer, 1x128 groups (row-wise) and/or 128x1 groups along

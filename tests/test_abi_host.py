@@ -197,3 +197,20 @@ def test_swiglu_quantize_rejections(lib):
     assert q(P(MIS), 256, 128, 1, P(A16), P(A16), None, None, S) == ALIGN
     assert q(P(A16), 0, 128, 3, None, None, None, None, S) == OK
     assert lib.fp8_selftest_silu_bf16(None, S) == NULL
+
+
+def test_split_threshold_setter(lib):
+    assert lib.fp8_set_gemm_split_min_work(-1) == SHAPE
+    assert lib.fp8_set_gemm_split_min_work(0) == OK
+    assert lib.fp8_set_gemm_split_min_work(fp8.GEMM_SPLIT_MIN_WORK_DEFAULT) == OK
+
+
+def test_binding_constants_match_the_header():
+    import re
+
+    from blockwise_fp8_pretraining_b200 import build
+
+    text = open(build.HEADER).read()
+    defines = dict(re.findall(r"#define\s+(FP8_\w+)\s+(\d+)", text))
+    assert int(defines["FP8_MAX_CONTRACTION_FPROP"]) == fp8.MAX_CONTRACTION_FPROP
+    assert int(defines["FP8_GEMM_SPLIT_MIN_WORK_DEFAULT"]) == fp8.GEMM_SPLIT_MIN_WORK_DEFAULT

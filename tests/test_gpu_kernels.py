@@ -23,7 +23,12 @@ def _device():
         pytest.skip("no CUDA device")
     fp8.load()
     fp8.fp8_clear_error()
+    # The shapes here are small: let the split schedule apply to them too
+    # whenever a workspace is given (its least-work threshold would keep
+    # most of them whole).
+    fp8.fp8_set_gemm_split_min_work(0)
     yield
+    fp8.fp8_set_gemm_split_min_work(fp8.GEMM_SPLIT_MIN_WORK_DEFAULT)
     assert fp8.fp8_get_error() == 0
 
 

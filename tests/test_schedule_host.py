@@ -13,6 +13,9 @@ Invariants the kernel relies on:
     loop skips pairs whose split range is empty);
   * without a workspace, with fewer than 32 slabs per tile, or when the last
     wave is at least 95% full, tiles are whole and assigned round-robin.
+The invariants are checked with the least-work threshold at 0, so that the
+split applies to the small shapes too; the default threshold is checked
+separately.
 """
 import pytest
 
@@ -43,6 +46,13 @@ def lib():
 
     build.build()
     return fp8.load()
+
+
+@pytest.fixture(autouse=True)
+def _split_everywhere(lib):
+    fp8.fp8_set_gemm_split_min_work(0)
+    yield
+    fp8.fp8_set_gemm_split_min_work(fp8.GEMM_SPLIT_MIN_WORK_DEFAULT)
 
 
 @pytest.mark.parametrize("split", [False, True])
@@ -121,3 +131,21 @@ def test_partial_last_waves_are_balanced(lib, M, N, K):
 def test_schedule_rejects_bad_sizes(lib):
     with pytest.raises(fp8.Fp8Error):
         fp8.fp8_selftest_gemm_schedule(100, 128, 128, PAIRS, True)
+
+
+@pytest.mark.parametrize("M,N,K,splits", [
+    (12288, 2048, 8192, True),      # gate_up wgrad: 332 units per pair
+    (8192, 2048, 12288, True),      # gate_up dgrad: 332
+    (8192, 2048, 6144, True),       # down fprop: 166
+    (2048, 6144, 8192, True),       # down wgrad: 166
+    (4096, 2048, 8192, False),      # qkv wgrad: 111
+    (8192, 2048, 4096, False),      # qkv dgrad: 111
+    (2048, 2048, 8192, False),      # o_proj wgrad: 55
+    (1280, 2304, 4096, False),
+])
+def test_default_least_work_keeps_short_gemms_whole(lib, M, N, K, splits):
+    fp8.fp8_set_gemm_split_min_work(fp8.GEMM_SPLIT_MIN_WORK_DEFAULT)
+    segs = fp8.fp8_selftest_gemm_schedule(M, N, K, PAIRS, True)
+    assert any(kb0 > 0 for _, _, kb0, _, _, _ in segs) == splits
+    fp8.fp8_set_gemm_split_min_work(tiles_of(M, N) * (K // 128) // PAIRS + 1)
+    assert all(kb0 == 0 for _, _, kb0, _, _, _ in fp8.fp8_selftest_gemm_schedule(M, N, K, PAIRS, True))
