@@ -317,13 +317,52 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
         if (__syncthreads_or(!ok)) break;
 
         if (SWIGLU) {
-            // ---- h over the gate tile (same swizzled layout as the up tile)
+            // ---- h over the gate tile (same swizzled layout as the up tile).
+            // Thread t forms chunks t + 256 j (8 elements each).  Elements
+            // whose silu rounding the FP32 path cannot decide (a fraction of
+            // a percent) keep their g and a bit in slow_bits; afterwards each
+            // warp deals its own out to its lanes for the FP64 path, so the
+            // hot loop has no call in it and no lane runs FP64 alone.
             uint8_t* gbuf = smem + (b ? L::OFF_IN1 : L::OFF_IN0);
+            uint64_t slow_bits = 0;              // bit 8 j + e: element e of chunk t + 256 j
 #pragma unroll 2
-            for (int c = t; c < 2 * tile::BOX_BYTES / 16; c += tile::THREADS) {
+            for (int j = 0; j < 2 * tile::BOX_BYTES / 16 / tile::THREADS; ++j) {
+                const int c = t + j * tile::THREADS;
                 const uint4 g = *reinterpret_cast<const uint4*>(gbuf + 16 * c);
                 const uint4 u = *reinterpret_cast<const uint4*>(gbuf + 2 * tile::BOX_BYTES + 16 * c);
-                *reinterpret_cast<uint4*>(gbuf + 16 * c) = swiglu8(g, u);
+                uint32_t slow = 0;
+                *reinterpret_cast<uint4*>(gbuf + 16 * c) = swiglu8_fast(g, u, slow);
+                slow_bits |= static_cast<uint64_t>(slow) << (8 * j);
+            }
+            __syncwarp();
+            const int cnt = __popcll(slow_bits);
+            int off = cnt;                       // inclusive, then exclusive, scan over the lanes
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, off, d);
+                if (lane >= d) off += v;
+            }
+            const int n_slow = __shfl_sync(0xffffffffu, off, 31);
+            off -= cnt;
+            for (int base = 0; base < n_slow; base += 32) {
+                const int k = base + lane;
+                int owner = 0;                   // the last lane whose range starts at or before k
+#pragma unroll
+                for (int step = 16; step > 0; step >>= 1) {
+                    const int o = __shfl_sync(0xffffffffu, off, owner + step);
+                    if (o <= k) owner += step;
+                }
+                const uint32_t m_lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(slow_bits), owner);
+                const uint32_t m_hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(slow_bits >> 32), owner);
+                const int r = k - __shfl_sync(0xffffffffu, off, owner);
+                if (k < n_slow) {
+                    uint64_t m = (static_cast<uint64_t>(m_hi) << 32) | m_lo;
+                    for (int i2 = 0; i2 < r; ++i2) m &= m - 1;     // drop the owner's first r elements
+                    const int bit = __ffsll(static_cast<long long>(m)) - 1;
+                    const int c = warp * 32 + owner + (bit >> 3) * tile::THREADS;
+                    swiglu_fix(reinterpret_cast<uint16_t*>(gbuf),
+                               reinterpret_cast<const uint16_t*>(gbuf + 2 * tile::BOX_BYTES), 8 * c + (bit & 7));
+                }
             }
             __syncthreads();
         }
