@@ -75,6 +75,10 @@ def _configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.orc_silu_bf16.argtypes = [ctypes.c_uint16]
     lib.orc_swiglu_bf16.restype = ctypes.c_int
     lib.orc_swiglu_bf16.argtypes = [p, i64, i64, p]
+    lib.orc_rmsnorm_rstd.restype = ctypes.c_int
+    lib.orc_rmsnorm_rstd.argtypes = [p, i64, i64, ctypes.c_float, p]
+    lib.orc_rmsnorm_apply.restype = ctypes.c_int
+    lib.orc_rmsnorm_apply.argtypes = [p, i64, i64, p, p, p]
     return lib
 
 
@@ -295,3 +299,30 @@ def swiglu_bf16(gate_up_bits: np.ndarray) -> np.ndarray:
     h = np.empty((rows, cols // 2), np.uint16)
     _check(_load().orc_swiglu_bf16(_ptr(x), rows, cols // 2, _ptr(h)), "swiglu_bf16")
     return h
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def rmsnorm_rstd(x_bits: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """r = fp32(1 / sqrt(mean(x^2) + eps)) per row of a bfloat16 [rows, cols]
+    (uint16 bits), the sum of squares in double."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = x.shape
+    r = np.empty(rows, np.float32)
+    _check(_load().orc_rmsnorm_rstd(_ptr(x), rows, cols, float(eps), _ptr(r)), "rmsnorm_rstd")
+    return r
+
+
+def rmsnorm_apply(x_bits: np.ndarray, r: np.ndarray, gamma_bits: np.ndarray) -> np.ndarray:
+    """y = bf16(gamma * bf16(fp32(x * r))) for x [rows, cols] (bfloat16
+    bits), r [rows] (float32) and gamma [cols] (bfloat16 bits).  Returns
+    uint16 bits [rows, cols]."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = x.shape
+    r = _c(r, np.float32)
+    g = _c(gamma_bits, np.uint16)
+    if r.shape != (rows,) or g.shape != (cols,):
+        raise ValueError("r must be [rows] and gamma [cols]")
+    y = np.empty((rows, cols), np.uint16)
+    _check(_load().orc_rmsnorm_apply(_ptr(x), rows, cols, _ptr(r), _ptr(g), _ptr(y)), "rmsnorm_apply")
+    return y

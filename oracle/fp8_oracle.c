@@ -546,3 +546,72 @@ int orc_swiglu_bf16(const uint16_t *gate_up, int64_t rows, int64_t ffn,
     }
     return bad ? -2 : 0;
 }
+
+/* -------------------------------------------------------------- RMSNorm
+ *
+ * The Qwen3-1.7B configuration (friendli.ai model card, model property
+ * table; the card's export class is Qwen3ForCausalLM) normalizes the input
+ * of the attention and feed-forward blocks with RMSNorm.  The linear
+ * layers' X is its BF16 output (training-setup paragraph: activations stay
+ * BF16), so a quantizer fused into the norm has to reproduce
+ *
+ *   r    = 1 / sqrt(mean_k x[k]^2 + eps)          per row, rounded to FP32
+ *   t[k] = fp32(x[k] * r)                         one FP32 multiply
+ *   y[k] = bf16(gamma[k] * bf16(t[k]))            each rounding to nearest even
+ *
+ * (the order of the Transformers Qwen3 RMSNorm: normalize in FP32, round to
+ * the activation type, then scale by the BF16 weight).  r is split off as
+ * its own function: the fused quantizer takes it as an input, computed by
+ * the row reduction that precedes it.
+ */
+
+/* r[i] for each row of x [rows, cols]: the squares of bfloat16 values are
+ * exact in double and their sum is taken in double in index order (for the
+ * row lengths of the path its relative error is below 2^-40); the mean is
+ * that sum / cols, eps is added in double, and 1 / sqrt(.) is rounded once
+ * from double to FP32. */
+int orc_rmsnorm_rstd(const uint16_t *x, int64_t rows, int64_t cols, float eps,
+                     float *r)
+{
+    if (rows < 0 || cols <= 0 || !(eps >= 0.0f))
+        return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int64_t i = 0; i < rows; ++i) {
+        double sum = 0.0;
+        for (int64_t k = 0; k < cols; ++k) {
+            double v = (double)orc_bf16_to_float(x[i * cols + k]);
+            if (!isfinite(v))
+                bad = 1;
+            sum += v * v;
+        }
+        double ms = sum / (double)cols + (double)eps;
+        r[i] = (float)(1.0 / sqrt(ms));
+    }
+    return bad ? -2 : 0;
+}
+
+/* y [rows, cols] = bf16(gamma * bf16(fp32(x * r))) with r per row (FP32)
+ * and gamma [cols] (bfloat16).  The FP32 product is a C float multiply
+ * (one IEEE rounding); the product of two bfloat16 values is exact in
+ * double, so each bfloat16 result has one rounding. */
+int orc_rmsnorm_apply(const uint16_t *x, int64_t rows, int64_t cols,
+                      const float *r, const uint16_t *gamma, uint16_t *y)
+{
+    if (rows < 0 || cols < 0)
+        return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int64_t k = 0; k < cols; ++k) {
+            float xf = orc_bf16_to_float(x[i * cols + k]);
+            float gf = orc_bf16_to_float(gamma[k]);
+            if (!isfinite(xf) || !isfinite(gf) || !isfinite(r[i]))
+                bad = 1;
+            volatile float t = xf * r[i];
+            double b = (double)orc_bf16_to_float(orc_bf16_from_double((double)t));
+            y[i * cols + k] = orc_bf16_from_double((double)gf * b);
+        }
+    }
+    return bad ? -2 : 0;
+}

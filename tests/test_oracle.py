@@ -676,3 +676,133 @@ def test_silu_rounding_margin_allows_fp64_evaluation():
         count += 1
     assert count > 9000
     assert smallest > 2e-9, smallest
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def _f32_nearest(v: Fraction):
+    """The float32 nearest to the positive rational v (ties to the even
+    significand), and whether v lies within 2^-38 (relative) of the midpoint
+    between it and a neighbour (where a double evaluation may decide
+    either way)."""
+    f = np.float32(float(v))
+    cands = {float(f), float(np.nextafter(f, np.float32(0))), float(np.nextafter(f, np.float32(np.inf)))}
+    ranked = sorted(cands, key=lambda c: (abs(Fraction(c) - v), int(np.float32(c).view(np.uint32)) & 1))
+    best, second = ranked[0], ranked[1]
+    gap = abs(abs(Fraction(second) - v) - abs(Fraction(best) - v))
+    return np.float32(best), gap < v * Fraction(1, 2 ** 38)
+
+
+def _rstd_exact(row_bits: np.ndarray, eps: np.float32):
+    import decimal
+
+    vals = [Fraction(float(v)) for v in oracle.bf16_to_float(row_bits).astype(np.float64)]
+    m = sum(v * v for v in vals) / len(vals) + Fraction(float(eps))
+    ctx = decimal.Context(prec=50)
+    d = ctx.divide(decimal.Decimal(1), ctx.sqrt(ctx.divide(decimal.Decimal(m.numerator), decimal.Decimal(m.denominator))))
+    return _f32_nearest(Fraction(d))
+
+
+def test_rmsnorm_rstd_closed_forms():
+    """Rows of one repeated value c: mean c^2, so r = 1 / |c| with eps = 0
+    (exact for powers of two); a zero row gives 1 / sqrt(eps)."""
+    for k in range(-6, 7):
+        c = np.float32(2.0 ** k)
+        row = to_bf16_bits(np.full((2, 384), c, np.float32))
+        row[1] |= 0x8000                             # the sign does not matter
+        assert list(oracle.rmsnorm_rstd(row, 0.0)) == [np.float32(2.0 ** -k)] * 2
+    three = to_bf16_bits(np.full((1, 256), 3.0, np.float32))
+    assert oracle.rmsnorm_rstd(three, 0.0)[0] == _f32_nearest(Fraction(1, 3))[0]
+    eps = np.float32(1e-6)
+    zero = np.zeros((1, 128), np.uint16)
+    assert oracle.rmsnorm_rstd(zero, float(eps))[0] == _rstd_exact(zero[0], eps)[0]
+    # one nonzero value x among n: mean x^2 / n
+    one = np.zeros((1, 512), np.uint16)
+    one[0, 37] = to_bf16_bits(np.float32([[8.0]]))[0, 0]
+    assert oracle.rmsnorm_rstd(one, 0.0)[0] == np.float32(np.sqrt(512.0) / 8.0)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_rmsnorm_rstd_against_exact_arithmetic(seed):
+    """Random rows (normal with x30 outlier channels, Student-t tails, tiny
+    magnitudes, 2048 and 6144 wide): the oracle's r equals the float32
+    nearest to the exact 1 / sqrt(mean + eps), computed in rational and
+    50-digit decimal arithmetic, except within 2^-38 of a rounding midpoint
+    where either neighbour is accepted."""
+    g = syn.generator(700 + seed)
+    eps = np.float32(1e-6)
+    rows = [syn.bf16_bits(syn.activation_bf16(3, 2048, 20, 30.0, g)),
+            syn.bf16_bits(syn.student_t_bf16((2, 6144), seed=seed)),
+            to_bf16_bits((np.random.default_rng(seed).standard_normal((2, 2048)) * 1e-3).astype(np.float32))]
+    checked = 0
+    for block in rows:
+        got = oracle.rmsnorm_rstd(block, float(eps))
+        for i in range(block.shape[0]):
+            want, near = _rstd_exact(block[i], eps)
+            if near:
+                assert abs(int(got[i].view(np.uint32)) - int(want.view(np.uint32))) <= 1
+            else:
+                assert got[i] == want, (i, got[i], want)
+            checked += 1
+    assert checked == 7
+
+
+def test_rmsnorm_apply_against_torch_and_exact_products():
+    """y = bf16(gamma * bf16(fp32(x * r))): the FP32 product and the first
+    rounding against torch's float32 multiply and bfloat16 cast, the second
+    against torch's bfloat16 multiply (computed in float32 and rounded),
+    which is exact wherever the float32 product is normal; subnormal
+    products against exact rational rounding."""
+    g = syn.generator(811)
+    rows, cols = 6, 384
+    x = syn.activation_bf16(rows, cols, 4, 30.0, g)
+    r = torch.exp(torch.empty(rows).uniform_(-20.0, 20.0, generator=g)).float()
+    gamma = (1.0 + 0.1 * torch.randn(cols, generator=g)).to(torch.bfloat16)
+    gamma[:5] = torch.tensor([0.0, -1.0, 2.0 ** -120, -3.5, 2.0 ** 60]).to(torch.bfloat16)
+    xb, gb = syn.bf16_bits(x), syn.bf16_bits(gamma)
+    y = oracle.rmsnorm_apply(xb, r.numpy(), gb)
+    t = (x.float() * r[:, None]).to(torch.bfloat16)
+    prod = gamma.float()[None, :] * t.float()
+    normal = (prod.abs() >= 2.0 ** -126) | (prod == 0)
+    want = syn.bf16_bits(gamma[None, :] * t)
+    assert np.array_equal(y[normal.numpy()], want[normal.numpy()])
+    tb = syn.bf16_bits(t)
+    for i, k in zip(*np.nonzero(~normal.numpy())):
+        v = Fraction(float(oracle.bf16_to_float(gb[k:k + 1])[0])) * Fraction(float(oracle.bf16_to_float(tb[i, k:k + 1])[0]))
+        assert int(y[i, k]) == _bf16_rne_exact(v, v < 0), (i, k)
+    assert (~normal).sum() > 0                       # the subnormal case is exercised
+
+
+def test_rmsnorm_is_invariant_to_power_of_two_row_scaling():
+    """With eps = 0, scaling a row by 2^k scales r by 2^-k exactly, so the
+    normalized and scaled output is unchanged."""
+    g = syn.generator(919)
+    x = syn.bf16_bits(syn.activation_bf16(4, 256, 3, 30.0, g))
+    gamma = syn.bf16_bits((1.0 + 0.1 * torch.randn(256, generator=g)).to(torch.bfloat16))
+    base = oracle.rmsnorm_apply(x, oracle.rmsnorm_rstd(x, 0.0), gamma)
+    for k in (-5, 3, 11):
+        xs = to_bf16_bits(oracle.bf16_to_float(x) * np.float32(2.0 ** k))
+        assert np.array_equal(oracle.rmsnorm_apply(xs, oracle.rmsnorm_rstd(xs, 0.0), gamma), base), k
+
+
+def test_rmsnorm_apply_fp32_product_near_bfloat16_midpoints():
+    """x * r chosen to land within a few float32 units of bfloat16 rounding
+    midpoints, where the bfloat16 result depends on the one float32
+    rounding of the product: against torch's float32 multiply and casts."""
+    rng = np.random.default_rng(5)
+    rows, cols = 64, 128
+    x = to_bf16_bits((rng.uniform(1.0, 2.0, (rows, cols)) * np.where(rng.random((rows, cols)) < 0.5, -1, 1))
+                     .astype(np.float32))
+    xf = oracle.bf16_to_float(x).astype(np.float64)
+    # per row: a bfloat16 midpoint M near 1 (9 significant bits, odd last)
+    # and r = fp32(M / x[row, 0]), so x[row, 0] * r is within an ulp of M;
+    # the other columns land near other midpoints less tightly
+    mids = (256 + 2 * rng.integers(0, 128, rows) + 1) / 512.0
+    r = (mids / xf[:, 0]).astype(np.float32)
+    gamma = np.full(cols, 0x3F80, np.uint16)          # gamma = 1: y is the first rounding
+    y = oracle.rmsnorm_apply(x, r, gamma)
+    t = (torch.from_numpy(xf.astype(np.float32)) * torch.from_numpy(r)[:, None]).to(torch.bfloat16)
+    assert np.array_equal(y, syn.bf16_bits(t))
+    prod = (xf.astype(np.float32) * r[:, None]).astype(np.float64)
+    units = prod[:, 0] * 512.0                       # midpoints in [1/2, 1) are odd multiples of 2^-9
+    assert np.mean((np.abs(units - np.round(units)) < 1e-4) & (np.round(units) % 2 == 1)) > 0.9

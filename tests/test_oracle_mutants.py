@@ -95,6 +95,16 @@ MUTANTS = [
      "double v = dw_in[n * K + k];", "double v = dw_in[i * K + k];", None),
     ("main-gradient accumulation subtracts the product",
      "dw_out[i * K + k] = v + dw_out[i * K + k];", "dw_out[i * K + k] = v - dw_out[i * K + k];", None),
+    ("rmsnorm: mean over cols - 1",
+     "double ms = sum / (double)cols + (double)eps;", "double ms = sum / (double)(cols - 1) + (double)eps;", None),
+    ("rmsnorm: eps left out",
+     "double ms = sum / (double)cols + (double)eps;", "double ms = sum / (double)cols;", None),
+    ("rmsnorm: r from float32 square root and division",
+     "r[i] = (float)(1.0 / sqrt(ms));", "r[i] = 1.0f / sqrtf((float)ms);", None),
+    ("rmsnorm: gamma applied before the first bfloat16 rounding",
+     "double b = (double)orc_bf16_to_float(orc_bf16_from_double((double)t));", "double b = (double)t;", None),
+    ("rmsnorm: x divided by 1/r instead of multiplied by r",
+     "volatile float t = xf * r[i];", "volatile float t = xf / (1.0f / r[i]);", None),
 ]
 
 
