@@ -219,16 +219,36 @@ class Sweep:
 
 
 def extra_launches(sweep):
-    """Launches of the two kernels outside the step's sweep, on the step's own
+    """Launches of the kernels outside the step's sweep, on the step's own
     buffers (after it has run): the fused SwiGLU producer on every layer's
     gate_up fprop output (H's codes for the down projection without H in
-    memory) and the wgrad of every linear accumulated into FP32 main
-    gradients."""
+    memory); the RMSNorm row statistic and the fused RMSNorm producer on
+    every layer's qkv and gate_up input, taken as the norm's input (X's
+    codes without X in memory); and the wgrad of every linear accumulated
+    into FP32 main gradients."""
     import torch
 
     T = TOKENS
     P = lambda t: ctypes.c_void_p(t.data_ptr())
     out = []
+    if not hasattr(sweep, "norm_gamma"):
+        gen = torch.Generator(device=sweep.device)
+        gen.manual_seed(4321)
+        hidden = dict((name, k) for name, _, k in linear_shapes())["qkv"]
+        sweep.norm_gamma = (1.0 + 0.1 * torch.randn(hidden, generator=gen, device=sweep.device)).to(torch.bfloat16)
+        sweep.norm_rstd = torch.empty(T, dtype=torch.float32, device=sweep.device)
+    gam, rstd = sweep.norm_gamma, sweep.norm_rstd
+    for l in range(sweep.layers):
+        for name in ("qkv", "gate_up"):
+            per, sh = sweep.layer[l][name], sweep.shared[name]
+            k = per["x"].shape[1]
+            out.append(("rmsnorm_rstd", "fp8_rmsnorm_rstd",
+                        lambda s, per=per, k=k: (P(per["x"]), T, k, ctypes.c_float(1e-6), P(rstd), s),
+                        0.0, T * k * 2 + T * 4, f"{name} rmsnorm rstd"))
+            out.append(("rmsnorm_quant_fused", "fp8_rmsnorm_quantize_1x128",
+                        lambda s, per=per, sh=sh, k=k: (P(per["x"]), T, k, P(rstd), P(gam), 3, P(sh["xq"]),
+                                                        P(sh["sx"]), P(per["xqT"]), P(per["sxT"]), s),
+                        0.0, T * k * (2 + 1 + 1 + 8 / 128) + T * 4 + k * 2, f"{name} fused rmsnorm producer"))
     ffn = dict((name, n) for name, n, _ in linear_shapes())["gate_up"] // 2
     gu, dn = sweep.shared["gate_up"], sweep.shared["down"]
     for l in range(sweep.layers):
@@ -765,6 +785,13 @@ def main_ours(args, rank, world, local_rank):
             # an unfused SwiGLU kernel writes H in bf16 and the quantizer reads it back
             sq["hbm_bytes_saved_per_layer_vs_unfused"] = ffn_elems * 4
             sq["input"] = "each layer's gate_up fprop output [8192, 12288] (gate | up), both layouts out"
+        rq = extra.get("rmsnorm_quant_fused")
+        if rq:
+            rq["frac_of_hbm"] = round(rq["gbs"] / pk["hbm_gbs"], 4)
+            rq["input"] = ("each layer's qkv and gate_up input [8192, 2048] as RMSNorm's input (rstd from "
+                           "rmsnorm_rstd), both layouts out")
+            # unfused: the norm reads x and writes y, the quantizer reads y; fused: x is read twice
+            rq["hbm_bytes_saved_per_launch_vs_unfused"] = TOKENS * 2048 * 2
         oa = extra.get("gemm_outer_accum_f32")
         if oa:
             oa["note"] = "wgrad of every linear added into FP32 main gradients (vector-reduction epilogue)"

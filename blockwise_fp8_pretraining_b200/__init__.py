@@ -26,6 +26,8 @@ from ._abi import (  # noqa: F401
     fp8_last_cuda_error,
     fp8_quantize_act_1x128,
     fp8_quantize_weight_128x128,
+    fp8_rmsnorm_quantize_1x128,
+    fp8_rmsnorm_rstd,
     fp8_selftest_division,
     fp8_selftest_gemm_schedule,
     fp8_selftest_silu_bf16,

@@ -59,6 +59,8 @@ def load() -> ctypes.CDLL:
         "fp8_quantize_act_1x128": [p, i64, i64, i32, p, p, p, p, p],
         "fp8_quantize_weight_128x128": [p, i64, i64, p, p, p, p],
         "fp8_swiglu_quantize_1x128": [p, i64, i64, i32, p, p, p, p, p],
+        "fp8_rmsnorm_rstd": [p, i64, i64, ctypes.c_float, p, p],
+        "fp8_rmsnorm_quantize_1x128": [p, i64, i64, p, p, i32, p, p, p, p, p],
         "fp8_selftest_silu_bf16": [p, p],
         "fp8_block_gemm_fprop": [p, p, p, p, p, i64, i64, i64, p, sz, p],
         "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p, sz, p],
@@ -222,6 +224,58 @@ def fp8_swiglu_quantize_1x128(gate_up, mode=BOTH, q_row=None, s_row=None, q_colT
     _check(lib.fp8_swiglu_quantize_1x128(_ptr(gate_up), rows, ffn, int(mode), _ptr(q_row), _ptr(s_row),
                                          _ptr(q_colT), _ptr(s_col), _stream(stream)),
            "fp8_swiglu_quantize_1x128")
+    return outs
+
+
+def fp8_rmsnorm_rstd(x, eps=1e-6, rstd=None, stream=None):
+    """RMSNorm's rstd[i] = 1 / sqrt(mean(x[i]^2) + eps) (float32 [rows]) of a
+    bf16 x [rows, cols]."""
+    lib = load()
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    _want(x, torch.bfloat16, (rows, cols), "x")
+    given = rstd is not None
+    rstd = _out(rstd, torch.float32, (rows,), x.device, "rstd")
+    _launch_checks([("x", x), ("rstd", rstd)], stream)
+    if not given:
+        _record(stream, [rstd])
+    _check(lib.fp8_rmsnorm_rstd(_ptr(x), rows, cols, float(eps), _ptr(rstd), _stream(stream)), "fp8_rmsnorm_rstd")
+    return rstd
+
+
+def fp8_rmsnorm_quantize_1x128(x, rstd, gamma, mode=BOTH, q_row=None, s_row=None, q_colT=None, s_col=None,
+                               stream=None):
+    """Quantize y = bf16(gamma * bf16(x * rstd)) (RMSNorm's output; rstd
+    float32 [rows], gamma bf16 [cols]) of a bf16 x [rows, cols] without
+    forming y in memory.  Returns (q_row, s_row, q_colT, s_col) of y;
+    entries of a grouping the mode leaves out are None."""
+    lib = load()
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    _want(x, torch.bfloat16, (rows, cols), "x")
+    _want(rstd, torch.float32, (rows,), "rstd")
+    _want(gamma, torch.bfloat16, (cols,), "gamma")
+    dev = x.device
+    given = [t is not None for t in (q_row, s_row, q_colT, s_col)]
+    if mode & ROWWISE:
+        q_row = _out(q_row, torch.uint8, (rows, cols), dev, "q_row")
+        s_row = _out(s_row, torch.float32, (cols // 128, rows), dev, "s_row")
+    else:
+        q_row = s_row = None
+    if mode & COLWISE:
+        q_colT = _out(q_colT, torch.uint8, (cols, rows), dev, "q_colT")
+        s_col = _out(s_col, torch.float32, (rows // 128, cols), dev, "s_col")
+    else:
+        q_colT = s_col = None
+    outs = (q_row, s_row, q_colT, s_col)
+    _launch_checks([("x", x), ("rstd", rstd), ("gamma", gamma), ("q_row", q_row), ("s_row", s_row),
+                    ("q_colT", q_colT), ("s_col", s_col)], stream)
+    _record(stream, [t for t, g in zip(outs, given) if not g])
+    _check(lib.fp8_rmsnorm_quantize_1x128(_ptr(x), rows, cols, _ptr(rstd), _ptr(gamma), int(mode), _ptr(q_row),
+                                          _ptr(s_row), _ptr(q_colT), _ptr(s_col), _stream(stream)),
+           "fp8_rmsnorm_quantize_1x128")
     return outs
 
 

@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8blk.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("fp8blk.cu", "gemm.cuh", "quantize.cuh", "ptx.cuh", "swiglu.cuh")]
+SOURCES = [os.path.join(CSRC, f) for f in ("fp8blk.cu", "gemm.cuh", "quantize.cuh", "ptx.cuh", "swiglu.cuh", "rmsnorm.cuh")]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fp8blk.h")
 
 NVCC_FLAGS = [

@@ -172,19 +172,22 @@ fp8_status make_map_2d(CUtensorMap* map, CUtensorMapDataType type, int elem_byte
 
 std::atomic<int> g_tile_attr_done[kMaxDevices];
 
-// Persistent 128 x 128 tile quantizer (column-wise, both, weight blocks, or,
-// with SWIGLU, the SwiGLU product of a gate_up activation [rows, 2 * cols]).
-template <int MODE, bool SWIGLU>
+// Persistent 128 x 128 tile quantizer (column-wise, both, weight blocks;
+// with kProdSwiglu the SwiGLU product of a gate_up activation [rows, 2 *
+// cols], with kProdNorm the RMSNorm output of x given r and gamma).
+template <int MODE, int PROD>
 fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* s_row,
-                             uint8_t* qT, float* s_col, cudaStream_t stream) {
+                             uint8_t* qT, float* s_col, cudaStream_t stream, const float* norm_r = nullptr,
+                             const void* norm_gamma = nullptr) {
+    constexpr bool SWIGLU = PROD == kProdSwiglu;
     using L = tile::Layout<SWIGLU>;
     int dev = 0, sms = 0;
     fp8_status st = current_device(&dev);
     if (st != FP8_OK) return st;
     if ((st = sm_count(dev, &sms)) != FP8_OK) return st;
-    const int flag = 1 << (MODE + 4 * (SWIGLU ? 1 : 0));
+    const int flag = 1 << (MODE + 4 * PROD);
     if ((g_tile_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
-        const cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE, SWIGLU>,
+        const cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE, PROD>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    L::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(quantize)", e);
@@ -206,10 +209,10 @@ fp8_status launch_tile_quant(const void* x, int64_t rows, int64_t cols, uint8_t*
     const int64_t tiles = (rows / 128) * (cols / 128);
     const int64_t cap = static_cast<int64_t>(L::BLOCKS_PER_SM) * sms;
     const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
-    const cudaError_t e = launch_pdl(quant_tile_kernel<MODE, SWIGLU>, dim3(grid), dim3(tile::THREADS),
+    const cudaError_t e = launch_pdl(quant_tile_kernel<MODE, PROD>, dim3(grid), dim3(tile::THREADS),
                                      L::SMEM_BYTES, stream, mx, mq, mqt, rows, cols, s_row, s_col,
                                      qT != nullptr ? 1 : 0, g_wait_ns.load(std::memory_order_relaxed),
-                                     take_stall(2));
+                                     take_stall(2), norm_r, static_cast<const __nv_bfloat16*>(norm_gamma));
     if (e != cudaSuccess) return cuda_fail("tile quantize launch", e);
     return last_launch_status("tile quantize launch");
 }
@@ -396,8 +399,8 @@ fp8_status fp8_quantize_act_1x128(const void* x_bf16, int64_t rows, int64_t cols
         return last_launch_status("row-wise quantize launch");
     }
     if (mode == FP8_COLWISE)
-        return launch_tile_quant<kTileColwise, false>(x_bf16, rows, cols, nullptr, nullptr, q_colT, s_col, s);
-    return launch_tile_quant<kTileBoth, false>(x_bf16, rows, cols, q_row, s_row, q_colT, s_col, s);
+        return launch_tile_quant<kTileColwise, kProdPlain>(x_bf16, rows, cols, nullptr, nullptr, q_colT, s_col, s);
+    return launch_tile_quant<kTileBoth, kProdPlain>(x_bf16, rows, cols, q_row, s_row, q_colT, s_col, s);
 }
 
 fp8_status fp8_swiglu_quantize_1x128(const void* gate_up_bf16, int64_t rows, int64_t ffn, int mode,
@@ -415,10 +418,48 @@ fp8_status fp8_swiglu_quantize_1x128(const void* gate_up_bf16, int64_t rows, int
     if ((mode & FP8_COLWISE) && (!aligned16(q_colT) || !aligned16(s_col))) return FP8_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (mode == FP8_ROWWISE)
-        return launch_tile_quant<kTileRowwise, true>(gate_up_bf16, rows, ffn, q_row, s_row, nullptr, nullptr, s);
+        return launch_tile_quant<kTileRowwise, kProdSwiglu>(gate_up_bf16, rows, ffn, q_row, s_row, nullptr, nullptr, s);
     if (mode == FP8_COLWISE)
-        return launch_tile_quant<kTileColwise, true>(gate_up_bf16, rows, ffn, nullptr, nullptr, q_colT, s_col, s);
-    return launch_tile_quant<kTileBoth, true>(gate_up_bf16, rows, ffn, q_row, s_row, q_colT, s_col, s);
+        return launch_tile_quant<kTileColwise, kProdSwiglu>(gate_up_bf16, rows, ffn, nullptr, nullptr, q_colT, s_col, s);
+    return launch_tile_quant<kTileBoth, kProdSwiglu>(gate_up_bf16, rows, ffn, q_row, s_row, q_colT, s_col, s);
+}
+
+fp8_status fp8_rmsnorm_rstd(const void* x_bf16, int64_t rows, int64_t cols, float eps, float* rstd,
+                            void* stream) {
+    if (rows < 0 || cols < 0 || cols % 8 || rows > kMaxDim || cols > kMaxDim) return FP8_ERR_SHAPE;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return FP8_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    if (!x_bf16 || !rstd) return FP8_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(rstd)) return FP8_ERR_ALIGN;
+    const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+    const cudaError_t e = launch_pdl(rmsnorm_rstd_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                                     static_cast<const uint4*>(x_bf16), rows, cols, eps, rstd);
+    if (e != cudaSuccess) return cuda_fail("rmsnorm rstd launch", e);
+    return last_launch_status("rmsnorm rstd launch");
+}
+
+fp8_status fp8_rmsnorm_quantize_1x128(const void* x_bf16, int64_t rows, int64_t cols, const float* rstd,
+                                      const void* gamma_bf16, int mode, uint8_t* q_row, float* s_row,
+                                      uint8_t* q_colT, float* s_col, void* stream) {
+    if (mode != FP8_ROWWISE && mode != FP8_COLWISE && mode != FP8_BOTH) return FP8_ERR_MODE;
+    if (rows < 0 || cols < 0 || rows % 128 || cols % 128 || rows > kMaxDim || cols > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP8_OK;
+    if (!x_bf16 || !rstd || !gamma_bf16) return FP8_ERR_NULL;
+    if ((mode & FP8_ROWWISE) && (!q_row || !s_row)) return FP8_ERR_NULL;
+    if ((mode & FP8_COLWISE) && (!q_colT || !s_col)) return FP8_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(rstd) || !aligned16(gamma_bf16)) return FP8_ERR_ALIGN;
+    if ((mode & FP8_ROWWISE) && (!aligned16(q_row) || !aligned16(s_row))) return FP8_ERR_ALIGN;
+    if ((mode & FP8_COLWISE) && (!aligned16(q_colT) || !aligned16(s_col))) return FP8_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (mode == FP8_ROWWISE)
+        return launch_tile_quant<kTileRowwise, kProdNorm>(x_bf16, rows, cols, q_row, s_row, nullptr, nullptr, s,
+                                                          rstd, gamma_bf16);
+    if (mode == FP8_COLWISE)
+        return launch_tile_quant<kTileColwise, kProdNorm>(x_bf16, rows, cols, nullptr, nullptr, q_colT, s_col, s,
+                                                          rstd, gamma_bf16);
+    return launch_tile_quant<kTileBoth, kProdNorm>(x_bf16, rows, cols, q_row, s_row, q_colT, s_col, s, rstd,
+                                                   gamma_bf16);
 }
 
 fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k, uint8_t* wq,
@@ -428,7 +469,7 @@ fp8_status fp8_quantize_weight_128x128(const void* w_bf16, int64_t n, int64_t k,
     if (!w_bf16 || !wq || !sw) return FP8_ERR_NULL;
     if (!aligned16(w_bf16) || !aligned16(wq) || !aligned16(sw) || (wqT && !aligned16(wqT)))
         return FP8_ERR_ALIGN;
-    return launch_tile_quant<kTileWeight, false>(w_bf16, n, k, wq, nullptr, wqT, sw,
+    return launch_tile_quant<kTileWeight, kProdPlain>(w_bf16, n, k, wq, nullptr, wqT, sw,
                                           static_cast<cudaStream_t>(stream));
 }
 

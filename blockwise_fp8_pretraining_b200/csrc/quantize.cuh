@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "rmsnorm.cuh"
 #include "swiglu.cuh"
 
 namespace fp8blk {
@@ -174,9 +175,13 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(const uint4* __restr
 
 // ---------------------------------------------------------------- 128x128 tiles
 
-// kTileRowwise is used with the SwiGLU input stage only; plain row-wise
-// groups have the lighter quant_rowwise_kernel.
+// kTileRowwise is used with the SwiGLU and RMSNorm input stages only;
+// plain row-wise groups have the lighter quant_rowwise_kernel.
 enum TileMode : int { kTileColwise = 0, kTileBoth = 1, kTileWeight = 2, kTileRowwise = 3 };
+// What the tile kernel quantizes: its input as it is, the SwiGLU product of
+// a gate_up activation, or the RMSNorm output y of its input (with r per
+// row and gamma per column given).
+enum TileProducer : int { kProdPlain = 0, kProdSwiglu = 1, kProdNorm = 2 };
 
 namespace tile {
 constexpr int THREADS = 256;
@@ -220,7 +225,7 @@ __device__ __forceinline__ int sw128(int r, int chunk) { return r * 128 + ((chun
 //   kTileWeight  : 128 x 128 blocks: q_row = codes [rows, cols], s_col =
 //                  block scales [rows/128, cols/128], transposed codes
 //                  through tmQT when has_qT
-//   kTileRowwise : groups along rows only (SWIGLU only)
+//   kTileRowwise : groups along rows only (SwiGLU and RMSNorm producers)
 // SWIGLU: the quantized tensor is h = bf16(bf16(silu(gate)) * up) of a
 // gate_up activation [rows, 2 * cols] (gate = columns [0, cols), up =
 // [cols, 2 * cols)); each tile buffer receives the gate and the up tile of
@@ -230,12 +235,14 @@ __device__ __forceinline__ int sw128(int r, int chunk) { return r * 128 + ((chun
 //   [cols, rows], box 128 x 128.
 // Row pass: lanes l and l + 16 of warp w share row 16 w + l % 16, 64 columns each.
 // Column pass: thread owns columns 2p, 2p+1 over the 32 rows of quarter qq.
-template <int MODE, bool SWIGLU>
-__global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PER_SM)
+template <int MODE, int PROD>
+__global__ void __launch_bounds__(tile::THREADS, tile::Layout<PROD == kProdSwiglu>::BLOCKS_PER_SM)
     quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmQT, int64_t rows, int64_t cols,
                       float* __restrict__ s_row, float* __restrict__ s_col, int has_qT,
-                      uint64_t wait_ns, uint32_t stall_tx) {
+                      uint64_t wait_ns, uint32_t stall_tx, const float* __restrict__ norm_r,
+                      const __nv_bfloat16* __restrict__ norm_gamma) {
+    constexpr bool SWIGLU = PROD == kProdSwiglu;
     using L = tile::Layout<SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -363,6 +370,23 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<SWIGLU>::BLOCKS_PE
                     swiglu_fix(reinterpret_cast<uint16_t*>(gbuf),
                                reinterpret_cast<const uint16_t*>(gbuf + 2 * tile::BOX_BYTES), 8 * c + (bit & 7));
                 }
+            }
+            __syncthreads();
+        }
+
+        if (PROD == kProdNorm) {
+            // ---- y = bf16(gamma * bf16(x * r)) over the tile, in place.
+            // Chunk c of the buffer: box c / 1024, row (c / 8) % 128, and
+            // 16-byte chunk (c % 8) ^ (row % 8) of that box row.
+            uint8_t* xbuf = smem + (b ? L::OFF_IN1 : L::OFF_IN0);
+#pragma unroll 2
+            for (int j = 0; j < 2 * tile::BOX_BYTES / 16 / tile::THREADS; ++j) {
+                const int c = t + j * tile::THREADS;
+                const int row = (c >> 3) & 127;
+                const int col = (c >> 10) * 64 + (((c & 7) ^ (row & 7)) << 3);
+                const float rr = __ldg(norm_r + r0 + row);
+                const uint4 gv = __ldg(reinterpret_cast<const uint4*>(norm_gamma + c0 + col));
+                *reinterpret_cast<uint4*>(xbuf + 16 * c) = rmsnorm8(*reinterpret_cast<const uint4*>(xbuf + 16 * c), rr, gv);
             }
             __syncthreads();
         }

@@ -10,15 +10,15 @@
 // the unfused H, so both roundings have to be the correctly rounded ones.
 //
 // silu(g) for a bfloat16 g is rounded once, correctly, to bfloat16:
-//   * 2^-20 <= |g| < 4: FP32 evaluation g / (1 + e) with e = __expf(-g)
+//   * 2^-20 <= |g| <= 80: FP32 evaluation g / (1 + e) with e = __expf(-g)
 //     and the fast division __fdividef.  __expf is within 2 + 1.173 |g|
 //     units in the last place (CUDA's documented bound for the intrinsic),
 //     __fdividef within 2, and 1 + e rounds once, so the quotient is within
 //     (5 + 1.173 |g|) * 2^-23 of silu(g), relative; a float32 unit in the
 //     last place at the result is at least 2^-24 of it, so the error is
-//     below 2 (5 + 1.173 |g|) < 12 + 3 |g| < 24 units.  When the FP32 value
-//     lies more than 32 units (that bound plus a margin of 8) from every
-//     bfloat16 rounding midpoint, it rounds like the exact value.
+//     below 2 (5 + 1.173 |g|) < 12 + 3 |g| units.  When the FP32 value lies
+//     more than 23 + 3 floor|g| units (that bound plus a margin of 8) from
+//     every bfloat16 rounding midpoint, it rounds like the exact value.
 //     Otherwise (a fraction of a percent of inputs) the element is
 //     evaluated in FP64; the fused producer collects such elements and
 //     evaluates them after the tile's pass, spread over a warp's lanes.
@@ -29,11 +29,9 @@
 //   * 200 <= |g|: silu(g) is g itself to within e^-200 (relative), and g
 //     is a bfloat16 value, so the result is g (g > 0); for g < 0 it is
 //     below 200 e^-200, far below half the smallest bfloat16, so -0.
-//   * elsewhere (including 4 <= |g|, rare in activations, where a
-//     constant margin would no longer cover the FP32 error) FP64
-//     evaluation with exp_fp64 (relative error below 2^-46); from 2^-30 to
-//     200 silu(g) stays more than 2e-9 (relative) away from every bfloat16
-//     midpoint, so it rounds like the exact value.
+//   * elsewhere FP64 evaluation with exp_fp64 (relative error below
+//     2^-46); from 2^-30 to 200 silu(g) stays more than 2e-9 (relative)
+//     away from every bfloat16 midpoint, so it rounds like the exact value.
 // An exhaustive check over all 65,536 inputs (fp8_selftest_silu_bf16)
 // compares this function with the oracle's correctly rounded silu.
 //
@@ -107,14 +105,15 @@ __device__ __noinline__ uint32_t silu_bf16_slow(float g) {
 // The FP32 fast path alone: true, with the bits, when it decides the
 // rounding; false when the element needs silu_bf16_slow.
 __device__ __forceinline__ bool silu_bf16_fast(float g, uint32_t& bits) {
-    // 2^-20 <= |g| < 4, compared on the bit pattern of |g|
+    // 2^-20 <= |g| <= 80, compared on the bit pattern of |g|
     const uint32_t ab = __float_as_uint(g) & 0x7FFFFFFFu;
-    if (ab - 0x35800000u < 0x40800000u - 0x35800000u) {
+    if (ab - 0x35800000u <= 0x42A00000u - 0x35800000u) {
         const float q = __fdividef(g, 1.0f + __expf(-g));
         bits = bf16_rne_bits(q);
-        // decided unless the low 16 bits lie within 32 units of the
-        // midpoint 0x8000, i.e. in [0x7FE0, 0x8020]
-        return (__float_as_uint(q) & 0xFFFFu) - 0x7FE0u > 64u;
+        // decided unless the low 16 bits lie within `margin` units of the
+        // midpoint 0x8000
+        const uint32_t margin = 23u + 3u * static_cast<uint32_t>(__uint_as_float(ab));
+        return (__float_as_uint(q) & 0xFFFFu) - (0x8000u - margin) > 2u * margin;
     }
     return false;
 }

@@ -170,6 +170,47 @@ fp8_status fp8_swiglu_quantize_1x128(const void *gate_up_bf16, int64_t rows, int
                                      uint8_t *q_colT, float *s_col, void *stream);
 
 /*
+ * RMSNorm's row statistic: rstd[i] = 1 / sqrt(mean_k x[i, k]^2 + eps),
+ * with the sum of squares in FP64 and one rounding to FP32 (the correctly
+ * rounded value except within 2^-40 of a rounding midpoint, where it may be
+ * the neighbouring float).  Passage: Puro-2B-Base model card (friendli.ai),
+ * model property table (Qwen3-1.7B configuration, exported as
+ * Qwen3ForCausalLM, whose blocks normalize their input with RMSNorm; the
+ * Transformers default eps is 1e-6).
+ *
+ *   x_bf16 [rows, cols] bf16, 16-byte aligned; rows >= 0, cols >= 0 a
+ *          multiple of 8.
+ *   eps    >= 0, finite.
+ *   rstd   [rows] f32, 16-byte aligned.
+ * rows == 0 or cols == 0 is a no-op (pointers may then be NULL).
+ */
+fp8_status fp8_rmsnorm_rstd(const void *x_bf16, int64_t rows, int64_t cols, float eps,
+                            float *rstd, void *stream);
+
+/*
+ * Fused RMSNorm producer: y = bf16(gamma * bf16(fp32(x * rstd))) per
+ * element (each rounding to nearest even; the order of the Transformers
+ * Qwen3 RMSNorm: normalize in FP32, round to BF16, scale by the weight),
+ * quantized like fp8_quantize_act_1x128 quantizes a bf16 y, without writing
+ * y to memory.  Given the same rstd, the codes and scales equal those of
+ * quantizing the unfused y bit for bit.  Passage: Puro-2B-Base model card,
+ * model property table (Qwen3-1.7B configuration) and training-setup
+ * paragraph (blockwise E4M3 linear-layer GEMMs on BF16 activations).
+ *
+ *   x_bf16     [rows, cols] bf16, 16-byte aligned; rows, cols >= 0,
+ *              multiples of 128.
+ *   rstd       [rows] f32 (for example from fp8_rmsnorm_rstd), 16-byte
+ *              aligned.
+ *   gamma_bf16 [cols] bf16 norm weight, 16-byte aligned.
+ *   mode, q_row, s_row, q_colT, s_col: as fp8_quantize_act_1x128.
+ * rows == 0 or cols == 0 is a no-op (pointers may then be NULL).
+ */
+fp8_status fp8_rmsnorm_quantize_1x128(const void *x_bf16, int64_t rows, int64_t cols,
+                                      const float *rstd, const void *gamma_bf16, int mode,
+                                      uint8_t *q_row, float *s_row, uint8_t *q_colT,
+                                      float *s_col, void *stream);
+
+/*
  * Weight quantizer, 128x128 blocks.
  * Passage: Puro-2B-Base model card, training-setup paragraph (blockwise E4M3);
  * the 128x128 block follows the DeepSeek-V3 recipe the Puro-2B tech report

@@ -214,3 +214,22 @@ def test_binding_constants_match_the_header():
     defines = dict(re.findall(r"#define\s+(FP8_\w+)\s+(\d+)", text))
     assert int(defines["FP8_MAX_CONTRACTION_FPROP"]) == fp8.MAX_CONTRACTION_FPROP
     assert int(defines["FP8_GEMM_SPLIT_MIN_WORK_DEFAULT"]) == fp8.GEMM_SPLIT_MIN_WORK_DEFAULT
+
+
+def test_rmsnorm_rejections(lib):
+    r = lib.fp8_rmsnorm_rstd
+    assert r(P(A16), 256, 100, 1e-6, P(A16), S) == SHAPE                   # cols % 8
+    assert r(P(A16), 256, 128, -1.0, P(A16), S) == SHAPE                   # eps < 0
+    assert r(None, 256, 128, 1e-6, P(A16), S) == NULL
+    assert r(P(MIS), 256, 128, 1e-6, P(A16), S) == ALIGN
+    assert r(P(A16), 0, 128, 1e-6, None, S) == OK
+    q = lib.fp8_rmsnorm_quantize_1x128
+    a = [P(A16)] * 3
+    assert q(P(A16), 256, 128, P(A16), P(A16), 0, *a[:2], None, None, S) == MODE
+    assert q(P(A16), 100, 128, P(A16), P(A16), 1, *a[:2], None, None, S) == SHAPE
+    assert q(P(A16), 256, 100, P(A16), P(A16), 1, *a[:2], None, None, S) == SHAPE
+    assert q(P(A16), 256, 128, None, P(A16), 1, *a[:2], None, None, S) == NULL
+    assert q(P(A16), 256, 128, P(A16), None, 1, *a[:2], None, None, S) == NULL
+    assert q(P(A16), 256, 128, P(A16), P(A16), 2, None, None, P(A16), None, S) == NULL
+    assert q(P(A16), 256, 128, P(A16), P(MIS), 1, *a[:2], None, None, S) == ALIGN
+    assert q(P(A16), 0, 128, None, None, 3, None, None, None, None, S) == OK

@@ -20,6 +20,8 @@ Configurations:
                          (even layers with the split schedule, odd without)
   heavy tails            Student-t(3) with 0.1% of values x1e3, seeds 0..27,
                          quantizers in full
+  RMSNorm producer       the attention X as the norm's input: r within one
+                         float32 ulp, fused codes and scales bit for bit
 """
 import os
 
@@ -56,6 +58,33 @@ def test_attention_projections_fprop():
     check_weight(c["w_o"])
     check_fprop(c["x"], c["w_qkv"], None, "qkv fprop", ws=workspace())
     check_fprop(c["x"], c["w_o"], None, "o_proj fprop", ws=workspace())
+
+
+def test_rmsnorm_producer_on_the_attention_input():
+    """The attention configuration's X [8192, 2048] taken as RMSNorm's input
+    (gamma ~ N(1, 0.1), eps 1e-6): the GPU's r against the oracle's (equal
+    or one float32 ulp apart), and the fused producer's codes and scales,
+    given the oracle's r, bit for bit in full against quantizing
+    y = bf16(gamma * bf16(x * r))."""
+    c = syn.attention_projections(seed=0)
+    x = c["x"]
+    g = syn.generator(77)
+    gamma = (1.0 + 0.1 * torch.randn(x.shape[1], generator=g)).to(torch.bfloat16)
+    xb, gb = syn.bf16_bits(x), syn.bf16_bits(gamma)
+    r = oracle.rmsnorm_rstd(xb, 1e-6)
+    r_gpu = fp8.fp8_rmsnorm_rstd(x.to(dev()), 1e-6).cpu().numpy()
+    diff = np.abs(r_gpu.view(np.int32).astype(np.int64) - r.view(np.int32).astype(np.int64))
+    assert diff.max() <= 1 and (diff != 0).mean() < 0.01
+    q_row, s_row, q_colT, s_col = fp8.fp8_rmsnorm_quantize_1x128(
+        x.to(dev()), torch.from_numpy(r).to(dev()), gamma.to(dev()), fp8.BOTH)
+    torch.cuda.synchronize()
+    y = oracle.rmsnorm_apply(xb, r, gb)
+    q_o, s_o = oracle.quantize_act_rowwise(y)
+    assert_bits_equal(q_row, q_o, "norm row-wise codes")
+    assert_bits_equal(s_row, s_o, "norm row-wise scales")
+    q_o, s_o = oracle.quantize_act_colwise(y)
+    assert_bits_equal(q_colT, q_o, "norm column-wise codes")
+    assert_bits_equal(s_col, s_o, "norm column-wise scales")
 
 
 def test_attention_projections_backward():

@@ -501,3 +501,55 @@ def test_swiglu_quantize_matches_the_unfused_definition(rows, ffn, mode):
         q_o, s_o = oracle.quantize_act_colwise(h)
         assert_bits_equal(q_colT, q_o, "fused column-wise codes")
         assert_bits_equal(s_col, s_o, "fused column-wise scales")
+
+
+# ------------------------------------------------------------ RMSNorm producer
+
+def _norm_case(rows, cols, seed):
+    """x with outlier channels, zero and tiny rows; gamma around 1 with
+    zeros, negatives and magnitudes that make subnormal products."""
+    g = syn.generator(seed)
+    x = syn.activation_bf16(rows, cols, max(1, cols // 100), 30.0, g)
+    x[0] = 0.0                                           # r = 1 / sqrt(eps)
+    x[1] = x[1] * 1e-30                                  # tiny row, eps dominates
+    x[2, :] = 3.0                                        # constant row
+    gamma = (1.0 + 0.1 * torch.randn(cols, generator=g))
+    gamma[:6] = torch.tensor([0.0, -1.0, 2.0 ** -120, -2.0 ** -126, 4.0, 2.0 ** 40])
+    return x.to(torch.bfloat16), gamma.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (8, 2048), (300, 6144), (1, 8)])
+def test_rmsnorm_rstd_matches_the_oracle(rows, cols):
+    """The FP64 sum of squares in another order than the oracle's: equal, or
+    one float32 ulp apart where the value sits next to a rounding midpoint."""
+    x, _ = _norm_case(max(rows, 3), cols, rows + cols)
+    x = x[:rows].contiguous()
+    r = fp8.fp8_rmsnorm_rstd(x.to(dev()), 1e-6)
+    torch.cuda.synchronize()
+    want = oracle.rmsnorm_rstd(syn.bf16_bits(x), 1e-6)
+    got = r.cpu().numpy()
+    diff = np.abs(got.view(np.int32).astype(np.int64) - want.view(np.int32).astype(np.int64))
+    assert diff.max() <= 1, diff.max()
+    assert (diff != 0).mean() < 0.01
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (384, 2048)])
+@pytest.mark.parametrize("mode", [fp8.ROWWISE, fp8.COLWISE, fp8.BOTH])
+def test_rmsnorm_quantize_matches_the_unfused_definition(rows, cols, mode):
+    """Given the oracle's r, the fused producer's codes and scales equal the
+    oracle's quantization of y = bf16(gamma * bf16(x * r)), bit for bit."""
+    x, gamma = _norm_case(rows, cols, 3 * rows + cols + mode)
+    xb, gb = syn.bf16_bits(x), syn.bf16_bits(gamma)
+    r = oracle.rmsnorm_rstd(xb, 1e-6)
+    q_row, s_row, q_colT, s_col = fp8.fp8_rmsnorm_quantize_1x128(
+        x.to(dev()), torch.from_numpy(r).to(dev()), gamma.to(dev()), mode)
+    torch.cuda.synchronize()
+    y = oracle.rmsnorm_apply(xb, r, gb)
+    if mode & fp8.ROWWISE:
+        q_o, s_o = oracle.quantize_act_rowwise(y)
+        assert_bits_equal(q_row, q_o, "norm row-wise codes")
+        assert_bits_equal(s_row, s_o, "norm row-wise scales")
+    if mode & fp8.COLWISE:
+        q_o, s_o = oracle.quantize_act_colwise(y)
+        assert_bits_equal(q_colT, q_o, "norm column-wise codes")
+        assert_bits_equal(s_col, s_o, "norm column-wise scales")
