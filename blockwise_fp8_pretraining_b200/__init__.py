@@ -17,6 +17,7 @@ from ._abi import (  # noqa: F401
     fp8_block_gemm_fprop,
     fp8_block_gemm_wgrad,
     fp8_block_gemm_wgrad_accum_f32,
+    fp8_block_gemm_wgrad_reduce_scatter_f32,
     fp8_block_gemm_wgrad_static_ws,
     fp8_cast_e4m3_scaled,
     fp8_clear_error,
@@ -37,6 +38,7 @@ from ._abi import (  # noqa: F401
     fp8_set_wait_timeout_ns,
     fp8_status_string,
     fp8_swiglu_quantize_1x128,
+    exchange_shards,
     header_functions,
     lib_path,
     load,

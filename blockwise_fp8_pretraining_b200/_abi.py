@@ -66,6 +66,7 @@ def load() -> ctypes.CDLL:
         "fp8_block_gemm_dgrad": [p, p, p, p, p, i64, i64, i64, p, sz, p],
         "fp8_block_gemm_wgrad": [p, p, p, p, p, i64, i64, i64, p, sz, p],
         "fp8_block_gemm_wgrad_accum_f32": [p, p, p, p, p, i64, i64, i64, p, sz, p],
+        "fp8_block_gemm_wgrad_reduce_scatter_f32": [p, p, p, p, p, i32, i64, i64, i64, p, sz, p],
         "fp8_gemm_workspace_bytes": [p],
         "fp8_block_gemm_wgrad_static_ws": [p, p, p, p, p, i64, i64, i64, p],
         "fp8_get_error": [],
@@ -408,6 +409,58 @@ def fp8_block_gemm_wgrad_accum_f32(dyqT, sdyT, xqT, sxT, dw, stream=None, worksp
                                               N, K, M, *_workspace(workspace), _stream(stream)),
            "fp8_block_gemm_wgrad_accum_f32")
     return dw
+
+
+MAX_SHARDS = 8
+
+
+def fp8_block_gemm_wgrad_reduce_scatter_f32(dyqT, sdyT, xqT, sxT, shards, stream=None, workspace=None):
+    """dW = dY^T X of this rank's tokens, added in FP32 into the owners'
+    shards: rows [q N / R, (q + 1) N / R) of dW into shards[q], a float32
+    [N / R, K] tensor of rank q (this GPU's, or a peer's mapped into this
+    process, see exchange_shards).  After every rank's call and a
+    synchronization each shard holds its old contents plus the sum over
+    ranks.  Returns shards."""
+    lib = load()
+    N, M = dyqT.shape
+    K = xqT.shape[0]
+    R = len(shards)
+    if not 1 <= R <= MAX_SHARDS or N % R:
+        raise ValueError(f"need 1..{MAX_SHARDS} shards dividing N = {N}, got {R}")
+    _want(dyqT, torch.uint8, (N, M), "dyqT")
+    _want(sdyT, torch.float32, (M // 128, N), "sdyT")
+    _want(xqT, torch.uint8, (K, M), "xqT")
+    _want(sxT, torch.float32, (M // 128, K), "sxT")
+    for q, t in enumerate(shards):            # peers' shards may live on other devices
+        _want(t, torch.float32, (N // R, K), f"shards[{q}]")
+    _launch_checks([("dyqT", dyqT), ("sdyT", sdyT), ("xqT", xqT), ("sxT", sxT), ("workspace", workspace)], stream)
+    table = (ctypes.c_void_p * R)(*[t.data_ptr() for t in shards])
+    _check(lib.fp8_block_gemm_wgrad_reduce_scatter_f32(_ptr(dyqT), _ptr(sdyT), _ptr(xqT), _ptr(sxT),
+                                                       ctypes.cast(table, ctypes.c_void_p), R, N, K, M,
+                                                       *_workspace(workspace), _stream(stream)),
+           "fp8_block_gemm_wgrad_reduce_scatter_f32")
+    return shards
+
+
+def exchange_shards(local, group=None, share=None, rebuild=None):
+    """The shards of a data-parallel group as seen from this rank: every
+    rank passes its own main-gradient shard; returns the list in rank order,
+    this rank's own tensor at its place and the others mapped into this
+    process through CUDA IPC (torch's tensor sharing).  share(t) turns a
+    tensor into a picklable handle and rebuild(handle) maps one back; they
+    default to torch.multiprocessing's CUDA reductions."""
+    import torch.distributed as dist
+
+    if share is None or rebuild is None:
+        from torch.multiprocessing.reductions import reduce_tensor
+
+        share = share or (lambda t: reduce_tensor(t))
+        rebuild = rebuild or (lambda h: h[0](*h[1]))
+    world = dist.get_world_size(group)
+    me = dist.get_rank(group)
+    handles = [None] * world
+    dist.all_gather_object(handles, share(local), group=group)
+    return [local if q == me else rebuild(handles[q]) for q in range(world)]
 
 
 def fp8_block_gemm_wgrad_static_ws(dyqT, sdyT, xqT, sxT, dw=None, stream=None):

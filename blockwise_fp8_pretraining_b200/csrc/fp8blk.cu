@@ -56,7 +56,7 @@ inline uint32_t take_stall(int bit) {
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_gemm_attr_done[kMaxDevices];
-std::atomic<int> g_gemm_pairs[kMaxDevices][8];   // co-resident CTA pairs per kernel variant
+std::atomic<int> g_gemm_pairs[kMaxDevices][12];  // co-resident CTA pairs per kernel variant
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 
@@ -250,7 +250,7 @@ inline int dp_tiles_for(int64_t tiles, int pairs, int num_kb) {
 // must not exceed it, or the last pairs would wait for a second wave).
 template <int SCALE, int OUT, bool SPLIT>
 fp8_status gemm_pairs(int dev, int sms, int* pairs_out) {
-    constexpr int variant = SCALE + 2 * OUT + 4 * (SPLIT ? 1 : 0);
+    constexpr int variant = SCALE + 2 * OUT + 6 * (SPLIT ? 1 : 0);
     const int flag = 1 << variant;
     if ((g_gemm_attr_done[dev].load(std::memory_order_relaxed) & flag) == 0) {
         cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<SCALE, OUT, SPLIT>,
@@ -292,7 +292,9 @@ fp8_status launch_gemm(const uint8_t* a, const uint8_t* b, void* out, gemm::Para
     if ((st = make_operand_map(&mb, b, p.N, p.K, gemm::BN / 2)) != FP8_OK) return st;
     // (main-gradient mode writes through p.out_f32; the map still needs a
     // valid encoding)
-    if ((st = make_output_map(&mc, out, p.M, p.N, OUT == gemm::kOutAccF32)) != FP8_OK) return st;
+    if ((st = make_output_map(&mc, out, OUT == gemm::kOutAccF32Shards ? (p.shard_rows > 32 ? p.shard_rows : 32) : p.M, p.N,
+                              OUT != gemm::kOutBf16)) != FP8_OK)
+        return st;
     if (OUT == gemm::kOutAccF32) p.out_f32 = static_cast<float*>(out);
 
     p.tiles_m = static_cast<int>((p.M + 2 * gemm::BM - 1) / (2 * gemm::BM));
@@ -540,6 +542,26 @@ fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t* dyqT, const float* sdyT
     return launch_gemm<gemm::kScaleOuter, gemm::kOutAccF32>(dyqT, xqT, dw_f32, wgrad_params(sdyT, sxT, N, K, M),
                                                             workspace, workspace_bytes,
                                                             static_cast<cudaStream_t>(stream));
+}
+
+fp8_status fp8_block_gemm_wgrad_reduce_scatter_f32(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,
+                                                  const float* sxT, float* const* dw_shards, int nranks,
+                                                  int64_t N, int64_t K, int64_t M, void* workspace,
+                                                  size_t workspace_bytes, void* stream) {
+    if (!dims_ok_gemm(N, K, M, true)) return FP8_ERR_SHAPE;
+    if (nranks < 1 || nranks > gemm::kMaxShards || N % nranks) return FP8_ERR_SHAPE;
+    if (!dyqT || !sdyT || !xqT || !sxT || !dw_shards) return FP8_ERR_NULL;
+    if (!aligned16(dyqT) || !aligned16(sdyT) || !aligned16(xqT) || !aligned16(sxT) || !aligned16(workspace))
+        return FP8_ERR_ALIGN;
+    gemm::Params p = wgrad_params(sdyT, sxT, N, K, M);
+    for (int q = 0; q < nranks; ++q) {
+        if (!dw_shards[q]) return FP8_ERR_NULL;
+        if (!aligned16(dw_shards[q])) return FP8_ERR_ALIGN;
+        p.shards[q] = dw_shards[q];
+    }
+    p.shard_rows = N / nranks;
+    return launch_gemm<gemm::kScaleOuter, gemm::kOutAccF32Shards>(dyqT, xqT, dw_shards[0], p, workspace,
+                                                                  workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fp8_status fp8_block_gemm_wgrad_static_ws(const uint8_t* dyqT, const float* sdyT, const uint8_t* xqT,

@@ -112,7 +112,13 @@ static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzled stages m
 constexpr uint32_t IDESC = idesc_e4m3_f32(2 * BM, BN);
 
 enum ScaleMode : int { kScaleRowBlock = 0, kScaleOuter = 1 };
-enum OutMode : int { kOutBf16 = 0, kOutAccF32 = 1 };
+// kOutAccF32Shards: like kOutAccF32, but row r of the output is added to
+// the shard that owns it (rows [q * shard_rows, (q + 1) * shard_rows) in
+// shard q, each a row-major [shard_rows, N] FP32 array, possibly in another
+// GPU's memory mapped into this process): the data-parallel reduce-scatter
+// of a weight gradient done by the epilogue's vector reductions.
+enum OutMode : int { kOutBf16 = 0, kOutAccF32 = 1, kOutAccF32Shards = 2 };
+constexpr int kMaxShards = 8;
 
 // Sleep between polls (ns) of the waits that are not on the hand-off's
 // critical path: the operand producer runs STAGES slabs ahead and the scale
@@ -140,6 +146,8 @@ struct Params {
     int dp_tiles;
     float* ws_partial;
     int* ws_flags;
+    float* shards[kMaxShards];  // kOutAccF32Shards: the owners' arrays
+    int64_t shard_rows;
 };
 
 // The work of one CTA pair: first its share of whole tiles (tile = pair,
@@ -587,11 +595,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // position j ^ (r % 8)), then TMA stores of the two boxes.
             const int m_own = (sg.tile / p.tiles_n) * (2 * BM) + static_cast<int>(rank) * BM;
             const int col0 = (sg.tile % p.tiles_n) * BN + half * 128;
-            if (OUT == kOutAccF32 && col0 < p.N && m_own < p.M) {
+            if ((OUT == kOutAccF32 || OUT == kOutAccF32Shards) && col0 < p.N && m_own < p.M) {
                 // FP32 added to the array in memory straight from the
                 // registers: one vector reduction per 4 columns, so each
-                // element receives exactly one addition per call
-                float* dst = p.out_f32 + static_cast<int64_t>(m_own + quarter * 32 + lane) * p.N + col0;
+                // element receives exactly one addition per call (per
+                // rank, when the shards gather several ranks' products)
+                const int64_t row = m_own + quarter * 32 + lane;
+                float* dst;
+                if (OUT == kOutAccF32Shards) {
+                    const int64_t owner = row / p.shard_rows;
+                    dst = p.shards[owner] + (row - owner * p.shard_rows) * p.N + col0;
+                } else {
+                    dst = p.out_f32 + row * p.N + col0;
+                }
 #pragma unroll
                 for (int j = 0; j < 128; j += 4)
                     red_add_v4_f32(dst + j, acc[j + 0], acc[j + 1], acc[j + 2], acc[j + 3]);

@@ -313,6 +313,38 @@ fp8_status fp8_block_gemm_wgrad_accum_f32(const uint8_t *dyqT, const float *sdyT
                                           void *stream);
 
 /*
+ * wgrad fused with the data-parallel reduce-scatter of the weight gradient,
+ * into FP32 main gradients: dW = dY^T X of this rank's tokens is added, as
+ * fp8_block_gemm_wgrad_accum_f32 adds it, straight into the shard of the
+ * rank that owns each row: rows [q N / nranks, (q + 1) N / nranks) of dW go
+ * to dw_shards[q], a row-major [N / nranks, K] FP32 array.  Shards of other
+ * GPUs are reached through peer mappings (CUDA IPC or peer access) with
+ * vector reductions over NVLink, issued tile by tile as each 256 x 256 tile
+ * of dW completes, so the transfer overlaps the GEMM.  When every rank of a
+ * data-parallel group has made this call on its own tokens, and the group
+ * has synchronized, shard q holds its previous contents plus the sum over
+ * ranks: the reduce-scatter.  Additions from different ranks meet in
+ * arbitrary order (each is one FP32 rounding).  Passage: Puro-2B-Base model
+ * card (friendli.ai), Phase 1 / Phase 2 setting table (data parallelism 12
+ * and 24) and training-setup paragraph (FP32 master state).
+ *
+ *   dyqT, sdyT, xqT, sxT, N, K, M, workspace, workspace_bytes - as
+ *            fp8_block_gemm_wgrad (M = this rank's tokens)
+ *   dw_shards  host array of nranks device pointers (this GPU's memory or
+ *            a peer's, mapped into this process), each 16-byte aligned
+ *   nranks   1 .. 8, dividing N
+ * The shards must not overlap the inputs; calls that add into the same
+ * shard on one GPU must be ordered (one stream), while calls of different
+ * ranks may run at the same time (the reductions are atomic).
+ */
+fp8_status fp8_block_gemm_wgrad_reduce_scatter_f32(const uint8_t *dyqT, const float *sdyT,
+                                                  const uint8_t *xqT, const float *sxT,
+                                                  float *const *dw_shards, int nranks,
+                                                  int64_t N, int64_t K, int64_t M,
+                                                  void *workspace, size_t workspace_bytes,
+                                                  void *stream);
+
+/*
  * wgrad for callers that cannot allocate device memory: the same GEMM as
  * fp8_block_gemm_wgrad with the split schedule, whose workspace here is a
  * fixed array inside the library instead of a buffer the caller passes.

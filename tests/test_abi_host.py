@@ -233,3 +233,20 @@ def test_rmsnorm_rejections(lib):
     assert q(P(A16), 256, 128, P(A16), P(A16), 2, None, None, P(A16), None, S) == NULL
     assert q(P(A16), 256, 128, P(A16), P(MIS), 1, *a[:2], None, None, S) == ALIGN
     assert q(P(A16), 0, 128, None, None, 3, None, None, None, None, S) == OK
+
+
+def test_wgrad_reduce_scatter_rejections(lib):
+    g = lib.fp8_block_gemm_wgrad_reduce_scatter_f32
+    a4 = [P(A16)] * 4
+    W = (None, 0)
+    table = (ctypes.c_void_p * 8)(*([A16] * 8))
+    T = ctypes.cast(table, ctypes.c_void_p)
+    assert g(*a4, T, 0, 256, 128, 128, *W, S) == SHAPE        # no ranks
+    assert g(*a4, T, 9, 256, 128, 128, *W, S) == SHAPE        # more than 8
+    assert g(*a4, T, 3, 256, 128, 128, *W, S) == SHAPE        # 3 does not divide 256
+    assert g(*a4, T, 2, 256, 128, 0, *W, S) == SHAPE          # no tokens
+    assert g(*a4, None, 2, 256, 128, 128, *W, S) == NULL
+    bad = (ctypes.c_void_p * 2)(A16, MIS)
+    assert g(*a4, ctypes.cast(bad, ctypes.c_void_p), 2, 256, 128, 128, *W, S) == ALIGN
+    null = (ctypes.c_void_p * 2)(A16, 0)
+    assert g(*a4, ctypes.cast(null, ctypes.c_void_p), 2, 256, 128, 128, *W, S) == NULL

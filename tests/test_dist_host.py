@@ -77,3 +77,37 @@ def test_reference_arm_nonzero_rank_exits_without_work():
                        env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def _exchange_main(rank, world, port, results):
+    import torch
+
+    import blockwise_fp8_pretraining_b200 as fp8
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        local = torch.full((2, 3), float(rank))
+        # stand-ins for CUDA IPC: the handle carries the rank and the values
+        shards = fp8.exchange_shards(local, share=lambda t: ("handle", rank, t.tolist()),
+                                     rebuild=lambda h: torch.tensor(h[2]) + 100 * (h[1] + 1))
+        results[rank] = ([s.tolist() for s in shards], [s is local for s in shards])
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shard_exchange_gloo_world2():
+    """exchange_shards gathers one handle per rank over the process group
+    and returns the shards in rank order: this rank's own tensor in its
+    place, every other rank's rebuilt from its handle."""
+    world = 2
+    with mp.get_context("spawn").Manager() as mgr:
+        results = mgr.dict()
+        mp.spawn(_exchange_main, args=(world, _free_port(), results), nprocs=world, join=True)
+        got = dict(results)
+    for rank in range(world):
+        values, is_local = got[rank]
+        assert is_local == [q == rank for q in range(world)]
+        for q in range(world):
+            want = float(q) if q == rank else float(q) + 100 * (q + 1)
+            assert values[q] == [[want] * 3] * 2

@@ -553,3 +553,42 @@ def test_rmsnorm_quantize_matches_the_unfused_definition(rows, cols, mode):
         q_o, s_o = oracle.quantize_act_colwise(y)
         assert_bits_equal(q_colT, q_o, "norm column-wise codes")
         assert_bits_equal(s_col, s_o, "norm column-wise scales")
+
+
+# -------------------------------------- fused wgrad + data-parallel reduce-scatter
+
+def _rank_inputs(N, K, M, seed):
+    g = syn.generator(seed)
+    dy = syn.normal_bf16((M, N), 1e-3, g)
+    x = syn.activation_bf16(M, K, 4, 30.0, g)
+    return dy, x
+
+
+@pytest.mark.parametrize("nranks,M,split", [(1, 256, False), (2, 256, False), (4, 4096, True), (8, 256, False)])
+def test_wgrad_reduce_scatter_into_emulated_ranks(nranks, M, split):
+    """R ranks' wgrad products, each over its own M tokens, added by the
+    fused epilogue into R FP32 shards (here all on this GPU; the addresses
+    are what differ from peers' shards).  Each shard ends as its start plus
+    the sum over ranks of its rows; against the oracle's FP64 sums, with each
+    call's 2e-3 S + 1e-6 plus half an FP32 ulp of the running value per
+    addition."""
+    N, K, d = 1024, 384, dev()
+    start = np.random.default_rng(nranks).normal(scale=0.01, size=(N, K)).astype(np.float32)
+    rows = N // nranks
+    shards = [torch.from_numpy(start[q * rows:(q + 1) * rows].copy()).to(d) for q in range(nranks)]
+    running = start.astype(np.float64)
+    tol = np.zeros((N, K))
+    for r in range(nranks):
+        dy, x = _rank_inputs(N, K, M, 5000 + 10 * nranks + r)
+        _, _, dyqT, sdyT = fp8.fp8_quantize_act_1x128(dy.to(d), fp8.COLWISE)
+        _, _, xqT, sxT = fp8.fp8_quantize_act_1x128(x.to(d), fp8.COLWISE)
+        fp8.fp8_block_gemm_wgrad_reduce_scatter_f32(dyqT, sdyT, xqT, sxT, shards,
+                                                    workspace=workspace() if split else None)
+        dyqT_o, sdyT_o = oracle.quantize_act_colwise(syn.bf16_bits(dy))
+        xqT_o, sxT_o = oracle.quantize_act_colwise(syn.bf16_bits(x))
+        running, bound = oracle.gemm_wgrad_accum(dyqT_o, sdyT_o, xqT_o, sxT_o, running)
+        tol += 2e-3 * bound + 1e-6 + 2.0 ** -24 * np.abs(running)
+    torch.cuda.synchronize()
+    got = np.concatenate([s.cpu().numpy() for s in shards]).astype(np.float64)
+    err = np.abs(got - running)
+    assert np.all(err <= tol), f"{int((err > tol).sum())} elements outside the bound"
