@@ -70,11 +70,11 @@ LAYERS = 28
 # Valid only for the kernels they were taken on; the profiles/ summaries give
 # the commands.  Remove an entry when its kernel changes.
 NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
-    "gemm_rowblock": (209136128.0, "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernel of commit 7466848"),
-    "gemm_outer": (177873152.0, "gate_up wgrad 12288x2048x8192, split schedule (algorithmic 167.8 MB plus the "
-                                "partial sums); kernel of commit 7466848"),
-    "quant_act": (360457472.0, "gate_up gradient 8192x12288, both layouts (algorithmic 408.9 MB); kernel of "
-                               "commit 4db2cd5"),
+    "gemm_rowblock": (204918016.0, "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernel of commit 64d796a"),
+    "gemm_outer": (176350976.0, "gate_up wgrad 12288x2048x8192, split schedule (algorithmic 167.8 MB plus the "
+                                "partial sums); kernel of commit 64d796a"),
+    "quant_act": (360666368.0, "gate_up gradient 8192x12288, both layouts (algorithmic 408.9 MB); kernel of "
+                               "commit 64d796a"),
 }
 
 
