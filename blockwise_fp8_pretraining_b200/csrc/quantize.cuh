@@ -276,13 +276,17 @@ __global__ void __launch_bounds__(tile::THREADS, tile::Layout<PROD == kProdSwigl
         }
     };
 
-    griddep_wait();                    // inputs of the preceding kernel are complete
-    if (t == 0) {
+    if (t == 0) {                      // set-up that reads nothing the preceding kernel writes
         mbar_init(bar0, 1);
         mbar_init(bar0 + 8, 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmQT);
+    }
+    griddep_wait();                    // inputs of the preceding kernel are complete
+    if (t == 0) {
         for (int j = 0; j < L::NBUF; ++j) {
             const int64_t tl = blockIdx.x + static_cast<int64_t>(j) * gridDim.x;
             if (tl < total) issue_load(tl, j);
