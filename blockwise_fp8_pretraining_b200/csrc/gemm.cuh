@@ -10,7 +10,14 @@
 // The result is either rounded to BF16 and stored, or (main-gradient mode)
 // added in FP32 to the FP32 array already in memory (vector reductions
 // straight from the registers, round-to-nearest-even; a subnormal sum may
-// be flushed to zero).
+// be flushed to zero), or added the same way into the data-parallel owners'
+// shards of that array (the reduce-scatter of a weight gradient).
+//
+// Work schedule (template parameter SPLIT): whole 256 x 256 tiles
+// round-robin over the CTA pairs, or, for long GEMMs whose last wave of
+// tiles would leave pairs idle, whole tiles for all waves but the last two
+// and then equal ranges of (tile, slab) units per pair, with FP32 partial
+// sums handed over through a workspace (see segment()).
 //
 // Structure: clusters of two CTAs (one per SM) compute 256 x 256 output
 // tiles; persistent, 384 threads (3 warpgroups) per CTA.
