@@ -73,8 +73,8 @@ NCU_TRAFFIC_BYTES_PER_LAUNCH: dict = {
     "gemm_rowblock": (204918016.0, "gate_up fprop 8192x12288x2048 (algorithmic 243.3 MB); kernel of commit 64d796a"),
     "gemm_outer": (176350976.0, "gate_up wgrad 12288x2048x8192, split schedule (algorithmic 167.8 MB plus the "
                                 "partial sums); kernel of commit 64d796a"),
-    "quant_act": (360666368.0, "gate_up gradient 8192x12288, both layouts (algorithmic 408.9 MB); kernel of "
-                               "commit 64d796a"),
+    "quant_act": (358906112.0, "gate_up gradient 8192x12288, both layouts (algorithmic 408.9 MB); kernel of "
+                               "commit 968e0c3"),
 }
 
 
