@@ -162,7 +162,7 @@ def test_clock_rejects_follows_the_timing_rules():
         assert bench.clock_rejects({"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap", bad]})
     # stuck well below max with nothing to explain it: a leftover clock lock
     assert bench.clock_rejects({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []})
-    # no sampler: nothing to judge by
+    # no sampler: no clock record to check
     assert not bench.clock_rejects({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]})
 
 
